@@ -1,0 +1,67 @@
+"""Each plausible mistake planted in a copy of the oracle source must fail
+at least one pin.  The mistakes are edits of the C source on the CPU; the
+committed oracle is untouched.  Every mistake keeps all memory accesses in
+bounds, so a mutant can only return wrong numbers, never crash."""
+
+import pytest
+
+import oracle
+import oracle_pins
+
+# (name, text in cca_oracle.c, replacement, which occurrence: 0 first, -1 all)
+MUTANTS = [
+    ("window counts self in w", "long lo = t - w;", "long lo = t - w + 1;", 0),
+    ("window not group aligned", "return (lo / g) * g;", "return lo;", 0),
+    ("pool scored by first query", "last = j * g + g - 1;", "last = j * g;", 0),
+    ("pool scale 1/d", "const double scale = 1.0 / sqrt((double)d);\n\n#pragma omp parallel num_threads(cca_oracle_threads())\n    {\n        double *s",
+     "const double scale = 1.0 / (double)d;\n\n#pragma omp parallel num_threads(cca_oracle_threads())\n    {\n        double *s", 0),
+    ("attention scale 1/d", "const double scale = 1.0 / sqrt((double)d);\n    for (long j = 0; j < nc; ++j) logit[j]",
+     "const double scale = 1.0 / (double)d;\n    for (long j = 0; j < nc; ++j) logit[j]", 0),
+    ("gqa sum not mean", "a[i] += s[i] / r;", "a[i] += s[i];", -1),
+    ("pool K with V", "ks += a[i] * Kh[(size_t)(first + i) * d + c];",
+     "ks += a[i] * Vh[(size_t)(first + i) * d + c];", 0),
+    ("pool transposed index", "Kh[(size_t)(first + i) * d + c]",
+     "Kh[(size_t)(first + c % g) * d + i % d]", 0),
+    ("one core token too many", "const long nc = ws / g, nl = t - ws + 1;\n                    const size_t kv",
+     "const long nc = ws / g + (ws < T - g ? 1 : 0), nl = t - ws + 1;\n                    const size_t kv", 0),
+    ("query misses itself", "const long nc = ws / g, nl = t - ws + 1;\n                    const size_t kv",
+     "const long nc = ws / g, nl = t - ws + (t > 0 ? 0 : 1);\n                    const size_t kv", 0),
+    ("raw weights misindexed", "out[c] += logit[nc + i] * vraw[i][c];",
+     "out[c] += logit[i] * vraw[i][c];", 0),
+    ("core values all from group 0", "out[c] += logit[j] * vcore[j][c];",
+     "out[c] += logit[j] * vcore[0][c];", 0),
+    ("softmax not normalised", "for (long i = 0; i < n; ++i) x[i] /= sum;",
+     "for (long i = 0; i < n; ++i) x[i] /= (sum + 1e-3);", 0),
+    ("append pools shifted group", "const long j = t / g, first = t - g + 1;",
+     "const long j = t / g, first = t - g;", 0),
+    ("append writes wrong core slot", "double *kc = c->k_core + (kv * c->core_cap + j) * d;",
+     "double *kc = c->k_core + (kv * c->core_cap + (j > 0 ? j - 1 : 0)) * d;", 0),
+    ("decode ring index off by one", "kp[nc + i] = c->k_tail + (kv * c->tail_cap +\n                                              p % c->tail_cap) * d;",
+     "kp[nc + i] = c->k_tail + (kv * c->tail_cap +\n                                              (p + 1) % c->tail_cap) * d;", 0),
+    ("capacity check off by one", "if (t / g >= c->core_cap) return CCA_ORACLE_ECAPACITY;",
+     "if (t / g > c->core_cap) return CCA_ORACLE_ECAPACITY;", 0),
+]
+
+
+def _mutate(src, old, new, which):
+    assert old in src, f"mutation anchor not found: {old!r}"
+    if which == -1:
+        return src.replace(old, new)
+    return src.replace(old, new, 1)
+
+
+@pytest.mark.parametrize("name,old,new,which", MUTANTS,
+                         ids=[m[0] for m in MUTANTS])
+def test_planted_mistake_is_caught(tmp_path, name, old, new, which):
+    src = _mutate(oracle.source(), old, new, which)
+    assert src != oracle.source()
+    mutant = oracle.build_variant(src, str(tmp_path / "libmutant.so"))
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mutant)
+        except AssertionError:
+            caught.append(pin.__name__)
+        except oracle.OracleError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin caught the planted mistake: {name}"
