@@ -1,0 +1,181 @@
+/*
+ * libcca: CCA-Attention (Core Context Aware attention) on NVIDIA B200
+ * (sm_100a), as a C ABI.
+ *
+ * The method is the one described in the write-up "ICML 2025 | 全局池化+局部
+ * 保留，CCA-Attention为LLM长文本建模带来突破性进展" of the paper "Core Context
+ * Aware Transformers for Long Context Language Modeling":
+ *
+ *  - globally-aware pooling (section 全局感知池化): the sequence is cut into
+ *    non-overlapping groups of g tokens; the query of each group's last
+ *    token scores the group's keys, softmax(q . k / sqrt(d)), and those
+ *    weights average the group's keys and values into one core key/value;
+ *  - locality-preserving module (section 局部保留模块): every token also sees
+ *    the raw keys/values of a window of at least w preceding tokens, aligned
+ *    to the group size;
+ *  - global-local fusion (section 全局-局部模块可微融合): one softmax over the
+ *    concatenation of the core and the raw keys;
+ *  - KV-cache support for decoding (section 基于 Triton 的底层加速).
+ *
+ * Definitions used by every call (r = Hq / Hkv; query head hq reads
+ * key/value head hq / r):
+ *   m          = floor(T / g) complete groups; group j = tokens jg..jg+g-1
+ *   ws(t)      = g * floor(max(t - w, 0) / g), start of t's local window
+ *   query t attends to core keys/values of groups j < ws(t) / g and to raw
+ *   keys/values ws(t)..t, all scaled by 1/sqrt(d), under one softmax.
+ *   Grouped-query attention (r > 1): each key/value head gets one core
+ *   key/value per group, weighted by the mean of its r query heads' softmax
+ *   vectors.
+ *
+ * Data: Q, K, V and raw cache rows are bf16; core keys/values (Kc, Vc and
+ * the cache's core slots) are fp16, whose 11 significant bits keep the
+ * error of the pooled rows of large keys well inside the attention's error
+ * budget.  All tensors are row-major and contiguous, layout [B, H, T, d]
+ * ("head-major"); d is 64 or 128.  Arithmetic is fp32 (scores, softmax,
+ * accumulation) with bf16 (raw keys) or fp16 (core keys) tensor-core
+ * operands.  Because core rows and the query copy used against them are
+ * fp16, input magnitudes must stay below 65504; larger values are clamped
+ * and reported as CCA_ERR_RANGE by cca_device_status().
+ *
+ * Memory: every pointer is a device pointer owned by the caller and
+ * borrowed for the call; the library allocates nothing.  Calls are
+ * asynchronous on the given stream (the CUDA runtime's cudaStream_t; 0 is
+ * the legacy default stream).  Outputs must not alias inputs.  Pointers
+ * must be 16-byte aligned.
+ *
+ * Errors: argument checks run on the host before any launch; a call that
+ * fails them returns a nonzero status and writes nothing.  CCA_ERR_CUDA
+ * reports a launch error.  Device-side waits are bounded: a wait that runs
+ * out records a timeout in a device status word and the kernel returns
+ * early; cca_device_status() reads and clears it (and the fp16 range flag).
+ */
+#ifndef CCA_H
+#define CCA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CCA_OK = 0,
+    CCA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or shape */
+    CCA_ERR_UNSUPPORTED = 2, /* d not 64/128, g or w beyond the limits     */
+    CCA_ERR_CAPACITY = 3,    /* cache has no room for the request          */
+    CCA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed          */
+    CCA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out         */
+    CCA_ERR_RANGE = 6        /* a value beyond the fp16 range was clamped  */
+} cca_status;
+
+/* Element type of an output that may be written in either precision. */
+typedef enum { CCA_BF16 = 0, CCA_F32 = 1 } cca_dtype;
+
+/* Largest group size the kernels accept. */
+#define CCA_MAX_G 256
+
+/*
+ * Decode cache (section 基于 Triton 的底层加速 says the kernel supports a KV
+ * cache; section 计算和存储效率对比 that it shrinks it).  It holds the core
+ * key/value of every completed group and the newest raw tokens in a ring:
+ *   k_core, v_core: fp16 [B, Hkv, core_cap, d]; slot j = group j
+ *   k_tail, v_tail: bf16 [B, Hkv, tail_cap, d]; token p in slot p % tail_cap
+ * tail_cap >= w + g keeps the whole local window of the newest token.
+ * All batch rows share one length `len` (tokens appended so far), which the
+ * host keeps in this struct.  The buffers belong to the caller.
+ */
+typedef struct {
+    void *k_core, *v_core;
+    void *k_tail, *v_tail;
+    int B, Hq, Hkv, d, g, w;
+    int64_t core_cap, tail_cap;
+    int64_t len;
+} cca_cache;
+
+/*
+ * Globally-aware pooling (section 全局感知池化).
+ *   Q [B, Hq, T, d], K and V [B, Hkv, T, d]  (bf16, read)
+ *   Kc, Vc [B, Hkv, m, d], m = floor(T / g)  (fp16, written)
+ * For each (b, kv head h, group j) the scores of the group's last query
+ * against the group's keys are soft-maxed (per query head, averaged over
+ * the r query heads of h) and pool that group's keys and values.  A trailing
+ * partial group is not pooled.  1 <= g <= CCA_MAX_G.
+ */
+cca_status cca_pool(const void *Q, const void *K, const void *V, void *Kc,
+                    void *Vc, int B, int Hq, int Hkv, int64_t T, int d, int g,
+                    cudaStream_t stream);
+
+/*
+ * Fused core + local attention for a whole sequence (sections 局部保留模块
+ * and 全局-局部模块可微融合).
+ *   Q [B, Hq, T, d], K, V [B, Hkv, T, d] (bf16), Kc, Vc [B, Hkv, m, d]
+ *   (fp16, from cca_pool), O [B, Hq, T, d] written in o_dtype (bf16 or
+ *   fp32).
+ * O[t] = softmax over { q_t . Kc[j] / sqrt(d) : j < ws(t)/g } and
+ * { q_t . K[i] / sqrt(d) : ws(t) <= i <= t } applied to [Vc ; V].
+ * Runs on tcgen05 tensor cores with TMA-staged tiles.
+ */
+cca_status cca_attn_prefill(const void *Q, const void *K, const void *V,
+                            const void *Kc, const void *Vc, void *O,
+                            cca_dtype o_dtype, int B, int Hq, int Hkv,
+                            int64_t T, int d, int g, int w,
+                            cudaStream_t stream);
+
+/*
+ * Fill a cache from a prefix of T tokens (Q, K, V as for cca_pool): pools
+ * every complete group into its core slot and copies the last
+ * min(T, tail_cap) raw tokens into their ring slots; sets c->len = T.
+ * CCA_ERR_CAPACITY if floor((T - 1) / g) >= core_cap.  The cache's shape
+ * fields (B, Hq, Hkv, d, g, w, core_cap, tail_cap) must be set.
+ */
+cca_status cca_cache_prefill(cca_cache *c, const void *Q, const void *K,
+                             const void *V, int64_t T, cudaStream_t stream);
+
+/*
+ * Append one token t = c->len per batch row: q_t [B, Hq, d], k_t, v_t
+ * [B, Hkv, d] (bf16).  k_t, v_t go to ring slot t % tail_cap; if the token
+ * completes group j = t / g ((t + 1) % g == 0), that group is pooled from
+ * the ring with the token's own queries (it is the group's last token) into
+ * core slot j.  On success c->len becomes t + 1.  CCA_ERR_CAPACITY (nothing
+ * written) if t / g >= core_cap.
+ */
+cca_status cca_cache_append(cca_cache *c, const void *q_t, const void *k_t,
+                            const void *v_t, cudaStream_t stream);
+
+/* Bytes of device workspace cca_attn_decode needs for this cache (for its
+ * current and any smaller length). */
+size_t cca_decode_workspace_bytes(const cca_cache *c);
+
+/*
+ * Attention of the newest token t = c->len - 1 over the cache: core slots
+ * j < ws(t)/g and ring slots of tokens ws(t)..t, one softmax.
+ *   q_t [B, Hq, d] (bf16), o_t [B, Hq, d] written in o_dtype.
+ * Split over key ranges; partial results go to `workspace` (device memory
+ * of at least cca_decode_workspace_bytes(c) bytes, 256-byte aligned, its
+ * contents need no initialisation), then a merge kernel combines them.
+ */
+cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
+                           cca_dtype o_dtype, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Synchronise `stream`, then report CCA_ERR_CUDA if a CUDA error is
+ * pending, CCA_ERR_TIMEOUT if any kernel of this library recorded a
+ * timed-out wait since the last call, CCA_ERR_RANGE if one clamped a value
+ * to the fp16 range, else CCA_OK.  The records are cleared.
+ */
+cca_status cca_device_status(cudaStream_t stream);
+
+/* Human-readable name of a status. */
+const char *cca_status_string(cca_status s);
+
+/* Library version, "major.minor.patch". */
+const char *cca_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* CCA_H */

@@ -1,0 +1,272 @@
+"""CCA-Attention on NVIDIA B200: Python binding of the C library libcca.
+
+Thin ctypes layer over ``include/cca.h``: it checks tensor devices, dtypes
+and layouts, allocates outputs with PyTorch when the caller passes none, and
+hands raw device pointers and the current CUDA stream to the library.  Every
+step of the computation runs in the library's CUDA kernels; there is no
+other code path.  If ``libcca.so`` is missing, every call raises.
+
+Build the library with ``python -m long_context_sparse_cca_b200.build``.
+
+Entry points (same names as the C ABI):
+    cca_pool, cca_attn_prefill, cca_cache_prefill, cca_cache_append,
+    cca_attn_decode, cca_decode_workspace_bytes, cca_device_status
+and the ``Cache`` class holding a decode cache's device buffers.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libcca.so")
+
+CCA_OK = 0
+CCA_ERR_INVALID_ARG = 1
+CCA_ERR_UNSUPPORTED = 2
+CCA_ERR_CAPACITY = 3
+CCA_ERR_CUDA = 4
+CCA_ERR_TIMEOUT = 5
+CCA_ERR_RANGE = 6
+CCA_BF16 = 0
+CCA_F32 = 1
+
+# Every symbol include/cca.h declares.
+EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
+           "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
+           "cca_device_status", "cca_status_string", "cca_version")
+
+
+class CCAError(RuntimeError):
+    """A nonzero status from libcca."""
+
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)}")
+
+
+class _CacheStruct(ctypes.Structure):
+    _fields_ = [("k_core", ctypes.c_void_p), ("v_core", ctypes.c_void_p),
+                ("k_tail", ctypes.c_void_p), ("v_tail", ctypes.c_void_p),
+                ("B", ctypes.c_int), ("Hq", ctypes.c_int), ("Hkv", ctypes.c_int),
+                ("d", ctypes.c_int), ("g", ctypes.c_int), ("w", ctypes.c_int),
+                ("core_cap", ctypes.c_int64), ("tail_cap", ctypes.c_int64),
+                ("len", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def lib():
+    """Load libcca.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(
+            f"libcca.so not found at {LIB_PATH}; build it with "
+            "`python -m long_context_sparse_cca_b200.build`")
+    L = ctypes.CDLL(LIB_PATH)
+    P, i, i64, st = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_int
+    CP = ctypes.POINTER(_CacheStruct)
+    L.cca_pool.argtypes = [P, P, P, P, P, i, i, i, i64, i, i, P]
+    L.cca_pool.restype = st
+    L.cca_attn_prefill.argtypes = [P, P, P, P, P, P, i, i, i, i, i64, i, i, i, P]
+    L.cca_attn_prefill.restype = st
+    L.cca_cache_prefill.argtypes = [CP, P, P, P, i64, P]
+    L.cca_cache_prefill.restype = st
+    L.cca_cache_append.argtypes = [CP, P, P, P, P]
+    L.cca_cache_append.restype = st
+    L.cca_decode_workspace_bytes.argtypes = [CP]
+    L.cca_decode_workspace_bytes.restype = ctypes.c_size_t
+    L.cca_attn_decode.argtypes = [CP, P, P, i, P, ctypes.c_size_t, P]
+    L.cca_attn_decode.restype = st
+    L.cca_device_status.argtypes = [P]
+    L.cca_device_status.restype = st
+    L.cca_status_string.argtypes = [i]
+    L.cca_status_string.restype = ctypes.c_char_p
+    L.cca_version.argtypes = []
+    L.cca_version.restype = ctypes.c_char_p
+    _lib = L
+    return L
+
+
+def status_string(status: int) -> str:
+    return lib().cca_status_string(int(status)).decode()
+
+
+def version() -> str:
+    return lib().cca_version().decode()
+
+
+def _check(status: int, what: str) -> None:
+    if status != CCA_OK:
+        raise CCAError(status, what)
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dev(t, name: str, dtype=None):
+    """Pointer of a contiguous CUDA tensor (None passes NULL)."""
+    if t is None:
+        return None
+    torch = _torch()
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    want = dtype or torch.bfloat16
+    if t.dtype != want:
+        raise ValueError(f"{name} must be {want}, got {t.dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _odtype(out_dtype) -> int:
+    torch = _torch()
+    if out_dtype in (torch.bfloat16, "bf16"):
+        return CCA_BF16
+    if out_dtype in (torch.float32, "f32", "fp32"):
+        return CCA_F32
+    raise ValueError(f"unsupported output dtype {out_dtype}")
+
+
+def cca_pool(Q, K, V, g: int, Kc=None, Vc=None, stream=None):
+    """Globally-aware pooling: Q [B,Hq,T,d], K/V [B,Hkv,T,d] (bf16, CUDA).
+
+    Returns (Kc, Vc) [B, Hkv, T // g, d] fp16.
+    """
+    torch = _torch()
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    m = T // g
+    if Kc is None:
+        Kc = torch.empty((B, Hkv, m, d), dtype=torch.float16, device=Q.device)
+    if Vc is None:
+        Vc = torch.empty((B, Hkv, m, d), dtype=torch.float16, device=Q.device)
+    if tuple(K.shape) != (B, Hkv, T, d) or tuple(V.shape) != (B, Hkv, T, d):
+        raise ValueError("K and V must be [B, Hkv, T, d]")
+    if tuple(Kc.shape) != (B, Hkv, m, d) or tuple(Vc.shape) != (B, Hkv, m, d):
+        raise ValueError("Kc and Vc must be [B, Hkv, T // g, d]")
+    _check(lib().cca_pool(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"),
+                          _dev(Kc, "Kc", torch.float16), _dev(Vc, "Vc", torch.float16),
+                          B, Hq, Hkv, T, d,
+                          int(g), _stream(stream)), "cca_pool")
+    return Kc, Vc
+
+
+def cca_attn_prefill(Q, K, V, Kc, Vc, g: int, w: int, O=None,
+                     out_dtype=None, stream=None):
+    """Fused core + local attention over the whole sequence.
+
+    Q [B,Hq,T,d], K/V [B,Hkv,T,d] (bf16), Kc/Vc [B,Hkv,T//g,d] (fp16).
+    Returns O [B, Hq, T, d] in ``out_dtype`` (bf16 default, or fp32).
+    """
+    torch = _torch()
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    if O is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        O = torch.empty((B, Hq, T, d), dtype=dt, device=Q.device)
+    od = _odtype(O.dtype)
+    if tuple(O.shape) != (B, Hq, T, d):
+        raise ValueError("O must be [B, Hq, T, d]")
+    _check(lib().cca_attn_prefill(
+        _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(Kc, "Kc", torch.float16),
+        _dev(Vc, "Vc", torch.float16), _dev(O, "O", O.dtype), od, B, Hq, Hkv, T, d, int(g),
+        int(w), _stream(stream)), "cca_attn_prefill")
+    return O
+
+
+class Cache:
+    """A decode cache: core slots of completed groups (fp16) plus a raw ring
+    of ``tail_cap`` tokens (bf16, default w + g), device buffers owned here."""
+
+    def __init__(self, B: int, Hq: int, Hkv: int, d: int, g: int, w: int,
+                 core_cap: int, tail_cap: Optional[int] = None, device="cuda"):
+        torch = _torch()
+        tail_cap = w + g if tail_cap is None else int(tail_cap)
+        kw = dict(dtype=torch.bfloat16, device=device)
+        kh = dict(dtype=torch.float16, device=device)
+        self.k_core = torch.zeros((B, Hkv, core_cap, d), **kh)
+        self.v_core = torch.zeros((B, Hkv, core_cap, d), **kh)
+        self.k_tail = torch.zeros((B, Hkv, tail_cap, d), **kw)
+        self.v_tail = torch.zeros((B, Hkv, tail_cap, d), **kw)
+        self.struct = _CacheStruct(self.k_core.data_ptr(), self.v_core.data_ptr(),
+                                   self.k_tail.data_ptr(), self.v_tail.data_ptr(),
+                                   B, Hq, Hkv, d, g, w, core_cap, tail_cap, 0)
+        self.workspace = None
+
+    @property
+    def len(self) -> int:
+        return int(self.struct.len)
+
+    @len.setter
+    def len(self, n: int) -> None:
+        self.struct.len = int(n)
+
+    def __getattr__(self, name):
+        if name in ("B", "Hq", "Hkv", "d", "g", "w", "core_cap", "tail_cap"):
+            return getattr(self.struct, name)
+        raise AttributeError(name)
+
+    def nbytes(self) -> int:
+        return sum(t.numel() * t.element_size() for t in
+                   (self.k_core, self.v_core, self.k_tail, self.v_tail))
+
+
+def cca_cache_prefill(cache: Cache, Q, K, V, stream=None) -> None:
+    """Fill ``cache`` from a prefix Q [B,Hq,T,d], K/V [B,Hkv,T,d]."""
+    T = Q.shape[2]
+    _check(lib().cca_cache_prefill(ctypes.byref(cache.struct), _dev(Q, "Q"),
+                                   _dev(K, "K"), _dev(V, "V"), T,
+                                   _stream(stream)), "cca_cache_prefill")
+
+
+def cca_cache_append(cache: Cache, q_t, k_t, v_t, stream=None) -> None:
+    """Append one token: q_t [B,Hq,d], k_t/v_t [B,Hkv,d] (bf16, CUDA)."""
+    _check(lib().cca_cache_append(ctypes.byref(cache.struct), _dev(q_t, "q_t"),
+                                  _dev(k_t, "k_t"), _dev(v_t, "v_t"),
+                                  _stream(stream)), "cca_cache_append")
+
+
+def cca_decode_workspace_bytes(cache: Cache) -> int:
+    return int(lib().cca_decode_workspace_bytes(ctypes.byref(cache.struct)))
+
+
+def cca_attn_decode(cache: Cache, q_t, o_t=None, out_dtype=None,
+                    workspace=None, stream=None):
+    """Attention of the newest token: q_t [B,Hq,d] -> o_t [B,Hq,d]."""
+    torch = _torch()
+    if o_t is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
+    od = _odtype(o_t.dtype)
+    nbytes = cca_decode_workspace_bytes(cache)
+    if workspace is None:
+        if cache.workspace is None or cache.workspace.numel() < nbytes:
+            cache.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8,
+                                          device=q_t.device)
+        workspace = cache.workspace
+    _check(lib().cca_attn_decode(
+        ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(o_t, "o_t", o_t.dtype),
+        od, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
+        _stream(stream)), "cca_attn_decode")
+    return o_t
+
+
+def cca_device_status(stream=None) -> int:
+    """Synchronise the stream; return the library's device status
+    (CCA_OK, CCA_ERR_TIMEOUT, CCA_ERR_RANGE or CCA_ERR_CUDA)."""
+    return int(lib().cca_device_status(_stream(stream)))

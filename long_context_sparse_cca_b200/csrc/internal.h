@@ -1,0 +1,62 @@
+// Host-side launchers of the CUDA kernels, called by the C ABI in api.cu
+// after it has checked every argument.  Each returns the launch's
+// cudaError_t.
+#pragma once
+
+#include <cuda_runtime_api.h>
+
+#include <cstddef>
+#include <cstdint>
+
+namespace cca {
+
+// Globally-aware pooling of all complete groups of Q/K/V [B,H,T,d] (bf16)
+// into Kc/Vc [B, Hkv, out_rows, d] (fp16; rows 0..floor(T/g)-1 written).
+cudaError_t launch_pool(const void *Q, const void *K, const void *V, void *Kc,
+                        void *Vc, int B, int Hq, int Hkv, int64_t T, int d,
+                        int g, int64_t out_rows, cudaStream_t s);
+
+// Copy raw tokens p in [p0, T) of K/V [B,Hkv,T,d] into ring slots
+// p % tail_cap of k_tail/v_tail [B,Hkv,tail_cap,d].
+cudaError_t launch_tail_fill(const void *K, const void *V, void *k_tail,
+                             void *v_tail, int B, int Hkv, int64_t T, int d,
+                             int64_t p0, int64_t tail_cap, cudaStream_t s);
+
+// Append token t (ring write; pool group t/g when (t+1) % g == 0).
+cudaError_t launch_append(const void *q_t, const void *k_t, const void *v_t,
+                          void *k_core, void *v_core, void *k_tail,
+                          void *v_tail, int B, int Hq, int Hkv, int d, int g,
+                          int64_t core_cap, int64_t tail_cap, int64_t t,
+                          cudaStream_t s);
+
+// Split-K decode over the cache for token t, then the merge.
+struct DecodePlan {
+    int64_t n_keys;   // keys of token t: core + raw
+    int64_t n_core;   // core keys
+    int64_t ws;       // window start
+    int chunk;        // keys per split
+    int nsplit;       // number of splits
+};
+DecodePlan decode_plan(int64_t t, int g, int w, int B, int Hkv);
+int decode_max_splits(int64_t core_cap, int64_t tail_cap);
+size_t decode_workspace_bytes(int B, int Hq, int d, int64_t core_cap,
+                              int64_t tail_cap);
+cudaError_t launch_decode(const void *k_core, const void *v_core,
+                          const void *k_tail, const void *v_tail,
+                          const void *q_t, void *o_t, bool o_f32,
+                          void *workspace, int B, int Hq, int Hkv, int d,
+                          int g, int w, int64_t core_cap, int64_t tail_cap,
+                          int64_t t, cudaStream_t s);
+
+// Fused core + local attention over a whole sequence (tcgen05 kernel).
+cudaError_t launch_prefill(const void *Q, const void *K, const void *V,
+                           const void *Kc, const void *Vc, void *O, bool o_f32,
+                           int B, int Hq, int Hkv, int64_t T, int d, int g,
+                           int w, cudaStream_t s);
+
+// Device status words (bits kStatusTimeout, kStatusRange): read and clear.
+cudaError_t prefill_status_read_clear(unsigned int *v);
+cudaError_t pool_status_read_clear(unsigned int *v);
+cudaError_t append_status_read_clear(unsigned int *v);
+
+}  // namespace cca

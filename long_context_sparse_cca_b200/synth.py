@@ -54,6 +54,14 @@ def bf16_bits_to_f64(b: np.ndarray) -> np.ndarray:
     return bf16_bits_to_f32(b).astype(np.float64)
 
 
+def f16_half_ulp(x: np.ndarray) -> np.ndarray:
+    """Half the spacing of fp16 numbers around |x| (11 significant bits;
+    spacing 2^-24 below the smallest normal 2^-14)."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -14)))
+    return np.ldexp(1.0, (e - 11).astype(np.int64))
+
+
 def bf16_half_ulp(x: np.ndarray) -> np.ndarray:
     """Half the spacing of bf16 numbers around |x| (the largest rounding error
     of a correctly rounded bf16 store of a value near x).

@@ -1,0 +1,132 @@
+"""The C-ABI library on the CPU: it builds, loads without a GPU, exports
+every entry point include/cca.h declares, and rejects bad arguments on the
+host before any launch (so these calls never reach the GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_sparse_cca_b200 as cca
+from long_context_sparse_cca_b200 import build as cca_build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x10000  # aligned, never dereferenced: every call below fails its checks
+
+
+@pytest.fixture(scope="module")
+def L():
+    cca_build.build()
+    return cca.lib()
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "cca.h")) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(cca_[a-z_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    declared = _declared()
+    assert len(declared) >= 9
+    for name in declared:
+        assert hasattr(L, name), name
+    assert sorted(declared) == sorted(cca.EXPORTS)
+
+
+def test_status_strings(L):
+    assert cca.status_string(cca.CCA_OK) == "CCA_OK"
+    assert cca.status_string(cca.CCA_ERR_TIMEOUT) == "CCA_ERR_TIMEOUT"
+    assert cca.status_string(99) == "CCA_ERR_UNKNOWN"
+    assert re.match(r"\d+\.\d+\.\d+", cca.version())
+
+
+def _pool(L, Q=FAKE, K=FAKE, V=FAKE, Kc=FAKE + 4096, Vc=FAKE + 8192, B=1,
+          Hq=2, Hkv=2, T=64, d=128, g=16):
+    P = ctypes.c_void_p
+    return L.cca_pool(P(Q), P(K), P(V), P(Kc), P(Vc), B, Hq, Hkv, T, d, g, None)
+
+
+def test_pool_argument_checks(L):
+    assert _pool(L, Q=0) == cca.CCA_ERR_INVALID_ARG
+    assert _pool(L, K=FAKE + 2) == cca.CCA_ERR_INVALID_ARG  # misaligned
+    assert _pool(L, d=96) == cca.CCA_ERR_UNSUPPORTED
+    assert _pool(L, Hq=3, Hkv=2) == cca.CCA_ERR_INVALID_ARG
+    assert _pool(L, g=0) == cca.CCA_ERR_INVALID_ARG
+    assert _pool(L, g=257) == cca.CCA_ERR_UNSUPPORTED
+    assert _pool(L, T=-1) == cca.CCA_ERR_INVALID_ARG
+    assert _pool(L, B=0) == cca.CCA_ERR_INVALID_ARG
+    # output overlapping an input
+    assert _pool(L, Kc=FAKE) == cca.CCA_ERR_INVALID_ARG
+    # no complete group: nothing to do, null pointers allowed
+    assert _pool(L, Q=0, K=0, V=0, Kc=0, Vc=0, T=15) == cca.CCA_OK
+
+
+def test_prefill_argument_checks(L):
+    P = ctypes.c_void_p
+
+    def call(O=FAKE + (1 << 24), od=0, d=128, T=300, g=16, w=64, Kc=FAKE + (1 << 20)):
+        return L.cca_attn_prefill(P(FAKE), P(FAKE), P(FAKE), P(Kc), P(Kc + 4096), P(O),
+                                  od, 1, 2, 2, T, d, g, w, None)
+
+    assert call(od=7) == cca.CCA_ERR_INVALID_ARG
+    assert call(O=0) == cca.CCA_ERR_INVALID_ARG
+    assert call(O=FAKE) == cca.CCA_ERR_INVALID_ARG  # O aliases Q
+    assert call(d=32) == cca.CCA_ERR_UNSUPPORTED
+    assert call(w=-1) == cca.CCA_ERR_INVALID_ARG
+    assert call(T=0, O=0) == cca.CCA_OK  # empty sequence
+    assert call(Kc=0) == cca.CCA_ERR_INVALID_ARG  # T // g > 0 needs Kc
+    assert call(Kc=FAKE + (1 << 20) + 8) == cca.CCA_ERR_INVALID_ARG  # misaligned
+
+
+def _cache(B=1, Hq=2, Hkv=2, d=128, g=16, w=64, core_cap=8, tail_cap=80, length=0,
+           ptrs=True):
+    base = FAKE if ptrs else 0
+    return cca._CacheStruct(base, base + (1 << 20), base + (2 << 20), base + (3 << 20),
+                            B, Hq, Hkv, d, g, w, core_cap, tail_cap, length)
+
+
+def test_cache_checks(L):
+    P = ctypes.c_void_p
+    c = _cache(tail_cap=79)  # below w + g
+    assert L.cca_cache_append(ctypes.byref(c), P(FAKE), P(FAKE), P(FAKE),
+                              None) == cca.CCA_ERR_INVALID_ARG
+    c = _cache(core_cap=2, length=32)  # token 32 belongs to group 2: no slot
+    assert L.cca_cache_append(ctypes.byref(c), P(FAKE), P(FAKE), P(FAKE),
+                              None) == cca.CCA_ERR_CAPACITY
+    assert c.len == 32
+    c = _cache(core_cap=2)
+    assert L.cca_cache_prefill(ctypes.byref(c), P(FAKE), P(FAKE), P(FAKE), 33,
+                               None) == cca.CCA_ERR_CAPACITY
+    assert c.len == 0
+    c = _cache(Hq=64, Hkv=2)
+    assert L.cca_decode_workspace_bytes(ctypes.byref(c)) == 0  # r > 16
+    c = _cache()
+    ws = L.cca_decode_workspace_bytes(ctypes.byref(c))
+    assert ws > 0
+    c.len = 0
+    assert L.cca_attn_decode(ctypes.byref(c), P(FAKE), P(FAKE + 4096), 0, P(FAKE),
+                             ws, None) == cca.CCA_ERR_INVALID_ARG  # empty cache
+    c.len = 10
+    assert L.cca_attn_decode(ctypes.byref(c), P(FAKE), P(FAKE + 4096), 0, P(FAKE),
+                             ws - 1, None) == cca.CCA_ERR_INVALID_ARG  # small ws
+    assert L.cca_attn_decode(ctypes.byref(c), P(FAKE), P(FAKE + 4096), 0,
+                             P(FAKE + 16), ws, None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_attn_decode(ctypes.byref(c), P(FAKE), P(FAKE + 4096), 3, P(FAKE),
+                             ws, None) == cca.CCA_ERR_INVALID_ARG  # dtype
+
+
+def test_workspace_grows_with_capacity(L):
+    a = _cache(core_cap=8)
+    b = _cache(core_cap=4096)
+    assert L.cca_decode_workspace_bytes(ctypes.byref(b)) > \
+        L.cca_decode_workspace_bytes(ctypes.byref(a))
+
+
+def test_binding_refuses_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(cca, "_lib", None)
+    monkeypatch.setattr(cca, "LIB_PATH", str(tmp_path / "missing.so"))
+    with pytest.raises(RuntimeError, match="libcca.so not found"):
+        cca.lib()
