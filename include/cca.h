@@ -175,6 +175,10 @@ const char *cca_status_string(cca_status s);
 /* Library version, "major.minor.patch". */
 const char *cca_version(void);
 
+/* Text of the CUDA error behind the calling thread's last CCA_ERR_CUDA
+ * ("no error" if there was none).  The string is static. */
+const char *cca_last_error(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -36,7 +36,7 @@ CCA_F32 = 1
 # Every symbol include/cca.h declares.
 EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
-           "cca_device_status", "cca_status_string", "cca_version")
+           "cca_device_status", "cca_status_string", "cca_version", "cca_last_error")
 
 
 class CCAError(RuntimeError):
@@ -89,6 +89,8 @@ def lib():
     L.cca_status_string.restype = ctypes.c_char_p
     L.cca_version.argtypes = []
     L.cca_version.restype = ctypes.c_char_p
+    L.cca_last_error.argtypes = []
+    L.cca_last_error.restype = ctypes.c_char_p
     _lib = L
     return L
 
@@ -101,8 +103,15 @@ def version() -> str:
     return lib().cca_version().decode()
 
 
+def last_error() -> str:
+    """CUDA error text behind this thread's last CCA_ERR_CUDA."""
+    return lib().cca_last_error().decode()
+
+
 def _check(status: int, what: str) -> None:
     if status != CCA_OK:
+        if status == CCA_ERR_CUDA:
+            what = f"{what} ({last_error()})"
         raise CCAError(status, what)
 
 

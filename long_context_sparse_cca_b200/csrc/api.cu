@@ -40,9 +40,13 @@ cca_status shape_status(int B, int Hq, int Hkv, int64_t T, int d, int g, int w)
     return CCA_OK;
 }
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
 cca_status from_cuda(cudaError_t e)
 {
-    return e == cudaSuccess ? CCA_OK : CCA_ERR_CUDA;
+    if (e == cudaSuccess) return CCA_OK;
+    g_last_cuda_error = e;
+    return CCA_ERR_CUDA;
 }
 
 cca_status cache_status(const cca_cache *c)
@@ -98,7 +102,7 @@ cca_status cca_attn_prefill(const void *Q, const void *K, const void *V, const v
         !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
         return CCA_ERR_INVALID_ARG;
     if (!any) return CCA_OK;
-    const int64_t n_items = ((T + 127) / 128) * int64_t(B) * Hq;
+    const int64_t n_items = ((T + 255) / 256) * int64_t(B) * Hq;
     if (n_items > INT32_MAX) return CCA_ERR_UNSUPPORTED;
     const size_t esz = o_dtype == CCA_F32 ? 4 : 2;
     const size_t out = size_t(B) * Hq * T * d * esz;
@@ -124,11 +128,11 @@ cca_status cca_cache_prefill(cca_cache *c, const void *Q, const void *K, const v
     if (any) {
         cudaError_t e = cca::launch_pool(Q, K, V, c->k_core, c->v_core, c->B, c->Hq,
                                          c->Hkv, T, c->d, c->g, c->core_cap, stream);
-        if (e != cudaSuccess) return CCA_ERR_CUDA;
+        if (e != cudaSuccess) return from_cuda(e);
         const int64_t p0 = T > c->tail_cap ? T - c->tail_cap : 0;
         e = cca::launch_tail_fill(K, V, c->k_tail, c->v_tail, c->B, c->Hkv, T, c->d, p0,
                                   c->tail_cap, stream);
-        if (e != cudaSuccess) return CCA_ERR_CUDA;
+        if (e != cudaSuccess) return from_cuda(e);
     }
     c->len = T;
     return CCA_OK;
@@ -147,7 +151,7 @@ cca_status cca_cache_append(cca_cache *c, const void *q_t, const void *k_t,
                                              c->k_tail, c->v_tail, c->B, c->Hq, c->Hkv,
                                              c->d, c->g, c->core_cap, c->tail_cap, t,
                                              stream);
-    if (e != cudaSuccess) return CCA_ERR_CUDA;
+    if (e != cudaSuccess) return from_cuda(e);
     c->len = t + 1;
     return CCA_OK;
 }
@@ -183,12 +187,13 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
 
 cca_status cca_device_status(cudaStream_t stream)
 {
-    if (cudaStreamSynchronize(stream) != cudaSuccess) return CCA_ERR_CUDA;
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return from_cuda(e);
     unsigned int a = 0, b = 0, c = 0;
-    if (cca::prefill_status_read_clear(&a) != cudaSuccess ||
-        cca::pool_status_read_clear(&b) != cudaSuccess ||
-        cca::append_status_read_clear(&c) != cudaSuccess)
-        return CCA_ERR_CUDA;
+    if ((e = cca::prefill_status_read_clear(&a)) != cudaSuccess ||
+        (e = cca::pool_status_read_clear(&b)) != cudaSuccess ||
+        (e = cca::append_status_read_clear(&c)) != cudaSuccess)
+        return from_cuda(e);
     const unsigned int st = a | b | c;
     if (st & cca::kStatusTimeout) return CCA_ERR_TIMEOUT;
     if (st & cca::kStatusRange) return CCA_ERR_RANGE;
@@ -210,5 +215,10 @@ const char *cca_status_string(cca_status s)
 }
 
 const char *cca_version(void) { return "0.1.0"; }
+
+const char *cca_last_error(void)
+{
+    return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 }  // extern "C"

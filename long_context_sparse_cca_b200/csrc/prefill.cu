@@ -10,20 +10,30 @@
 // MMAs with bf16 P; core tiles as fp16 x fp16 MMAs against an fp16 copy of
 // the Q tile, with fp16 P.
 //
-// Design (one persistent CTA per SM, 192 threads):
-//   warps 0-3  softmax: thread i owns query row i of the 128-row tile; makes
-//              the fp16 copy of Q; reads S from tensor memory, masks, online
-//              softmax (fp32, exp2, lazy rescale), writes P back into tensor
-//              memory over S, rescales O when its max moved, and runs the
-//              epilogue O / l.
-//   warp 4     TMA producer: Q tile, then per key tile a K tile and a V tile
-//              into multi-stage shared-memory rings (128-byte swizzle).
-//   warp 5     tcgen05 issuer: S = Q K^T (A, B from shared memory) into one of
-//              two S buffers in tensor memory; O += P V (A = P from tensor
-//              memory, B = V from shared memory).
-// Tensor memory: S0 [0,128), S1 [128,256), O [256, 256 + D) columns.
-// Work items are (query tile, batch, query head), heaviest (latest) query
-// tiles first, dealt round-robin to the CTAs.
+// Work item: a 256-row block of queries of one (batch, query head), split in
+// two 128-row halves A and B that share every K/V tile.  Its key tiles are
+// the local stream first (keys ws(t0) .. last row), then the core stream
+// (pooled keys 0 .. ws(last row)/g - 1); rows mask the keys they do not see.
+// Blocks are dealt round-robin to one persistent CTA per SM, latest blocks
+// (most core tiles) first.
+//
+// CTA of 320 threads (168 registers a thread: registers are booked for warps
+// in groups of four, so ten warps count as twelve):
+//   warps 0-3  softmax of half A, warps 4-7 softmax of half B: thread i owns
+//              query row i of its half; reads S from tensor memory, masks,
+//              online softmax (fp32; exp2 partly on the MUFU unit and partly
+//              as a polynomial on the FMA pipe; lazy rescale), writes P back
+//              into tensor memory over S, rescales O when its reference max
+//              moved, and runs the epilogue O / l.  At the switch from the
+//              local to the core stream each group turns its half of the Q
+//              tile from bf16 into fp16 in place.
+//   warp 8     TMA producer: the Q block, then per key tile one K and one V
+//              tile into multi-stage shared-memory rings (128-byte swizzle).
+//   warp 9     tcgen05 issuer, ping-pong between the halves:
+//              ... O_A += P_A V_{j-1}; S_A = Q_A K_j^T; O_B += P_B V_{j-1};
+//              S_B = Q_B K_j^T ...  (S from shared memory operands, P from
+//              tensor memory).
+// Tensor memory: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B after.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -38,45 +48,47 @@ __device__ unsigned int g_prefill_status;  // kStatusTimeout | kStatusRange
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr float kRescaleThreshold = 8.0f;         // log2 units
+constexpr float kRescaleThreshold = 8.0f;         // log2 units: P stays <= 256
+
+// Share of the exponentials computed on the FMA pipe: pairs i with
+// (i % 8) < kPolyPerEight of each 16-pair chunk of a row.
+constexpr int kPolyPerEight = 3;
+
+// 2^f on [-1/2, 1/2] by a degree-3 polynomial whose coefficients were fitted
+// for this kernel (Remez exchange on the relative error, weight 2^-f); max
+// relative error 7.5e-5, below half an fp16 spacing (a float32 replay of
+// these steps is checked against 2^y by the tests).
+constexpr float kP0 = 0.9999280571937561f;
+constexpr float kP1 = 0.6932609677314758f;
+constexpr float kP2 = 0.2426111251115799f;
+constexpr float kP3 = 0.0551716685295105f;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
 template <int D>
 struct Pf {
-    // 128 query rows per tile, 128 keys per tile
     static constexpr int NBOX = D / 64;          // 64-column swizzled boxes
     static constexpr int BOX_BYTES = 128 * 128;  // 128 rows x 128 bytes
-    static constexpr int TILE_BYTES = BOX_BYTES * NBOX;
+    static constexpr int TILE_BYTES = BOX_BYTES * NBOX;  // 128 rows x D
     static constexpr int KST = D == 128 ? 3 : 4;  // K ring stages
-    static constexpr int VST = D == 128 ? 2 : 3;  // V ring stages
-    static constexpr int OFF_Q = 0;                     // Q tile, bf16
-    static constexpr int OFF_QH = TILE_BYTES;           // Q tile, fp16 copy
+    static constexpr int VST = D == 128 ? 2 : 4;  // V ring stages
+    static constexpr int OFF_Q = 0;               // Q halves A, B (bf16, then fp16)
     static constexpr int OFF_K = 2 * TILE_BYTES;
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;  // + barriers + align slack
-    static constexpr uint32_t S_STRIDE = 128;  // S buffer b at column b * 128
-    static constexpr uint32_t O_COL = 256;
+    static constexpr uint32_t S_COL = 0;          // S of half h at h * 128
+    static constexpr uint32_t O_COL = 256;        // O of half h at 256 + h * D
     static constexpr uint32_t TMEM_COLS = 512;
+    static constexpr int THREADS = 320;
 };
 
 struct Params {
     int B, Hq, Hkv, r;
     int T, g, w, m;
-    int n_qtiles, n_items;
+    int n_blocks, n_items;
     float scale_log2;
     void *O;
     int o_f32;
-};
-
-// Geometry of one work item (query tile t0 .. tlast of one batch entry and
-// query head).  Its key tiles are the local stream first (raw keys
-// ws(t0) .. tlast, bf16), then the core stream (pooled keys 0 ..
-// ws(tlast)/g - 1, fp16).
-struct Geom {
-    int b, hq, h, t0, tlast;
-    int ws_lo, ws_hi;     // ws(t0), ws(tlast)
-    int nc_lo, nc_hi;     // core counts of the first / last row
-    int n_local, n_core_tiles, n_tiles;
 };
 
 __device__ __forceinline__ int ws_of(int t, int g, int w)
@@ -85,28 +97,32 @@ __device__ __forceinline__ int ws_of(int t, int g, int w)
     return (lo / g) * g;
 }
 
+// Geometry of one 256-row block.
+struct Geom {
+    int b, hq, h, t0, tlast;
+    int ws_lo;                 // ws(t0): first local key
+    int n_local, n_core_tiles, n_tiles;
+};
+
 __device__ __forceinline__ Geom geom(int item, const Params &p)
 {
     Geom G;
     const int bhq_count = p.B * p.Hq;
-    const int qt = p.n_qtiles - 1 - item / bhq_count;
+    const int blk = p.n_blocks - 1 - item / bhq_count;
     const int bhq = item - (item / bhq_count) * bhq_count;
     G.b = bhq / p.Hq;
     G.hq = bhq - G.b * p.Hq;
     G.h = G.hq / p.r;
-    G.t0 = qt * 128;
-    G.tlast = min(G.t0 + 127, p.T - 1);
+    G.t0 = blk * 256;
+    G.tlast = min(G.t0 + 255, p.T - 1);
     G.ws_lo = ws_of(G.t0, p.g, p.w);
-    G.ws_hi = ws_of(G.tlast, p.g, p.w);
-    G.nc_lo = G.ws_lo / p.g;
-    G.nc_hi = G.ws_hi / p.g;
-    G.n_core_tiles = (G.nc_hi + 127) / 128;
+    const int nc_hi = ws_of(G.tlast, p.g, p.w) / p.g;
+    G.n_core_tiles = (nc_hi + 127) / 128;
     G.n_local = (G.tlast - G.ws_lo + 1 + 127) / 128;
     G.n_tiles = G.n_local + G.n_core_tiles;
     return G;
 }
 
-// Key tile j of an item: stream and first key index.
 __device__ __forceinline__ bool tile_is_core(const Geom &G, int j) { return j >= G.n_local; }
 __device__ __forceinline__ int tile_key0(const Geom &G, int j)
 {
@@ -114,11 +130,13 @@ __device__ __forceinline__ int tile_key0(const Geom &G, int j)
 }
 
 struct Bars {
-    uint64_t q_full, q_empty, qh_full;
+    uint64_t q_full, q_empty, qloc_done;
+    uint64_t qh_full[2];
     uint64_t k_full[4], k_empty[4];
     uint64_t v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2];
-    uint64_t o_bar, o_empty, mma_done;
+    uint64_t o_bar[2], o_empty[2];
+    uint64_t mma_done;
     uint32_t tmem_base;
     int abort;  // set when any role gives up
     int never;  // stays 0: drain waits are bounded by time only
@@ -146,8 +164,135 @@ __device__ __forceinline__ bool lane_wait(uint64_t *bar, uint32_t parity, Bars *
     return ok;
 }
 
+// ------------------------------------------------------------ exp2 on pairs
+
+__device__ __forceinline__ float fmax3(float a, float b, float c)
+{
+    float d;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+    return d;
+}
+
+// 2^y for a pair, on the FMA pipe: y = n + f with n = rint(y) read from the
+// low mantissa bits of y + 1.5*2^23, f in [-1/2, 1/2] through the degree-3
+// polynomial, n added to the result's exponent field.  y is clamped to
+// >= -125 first, so the exponent field stays positive (2^-125 is far below
+// anything a row sum can notice; masked logits, -inf, land there).
+__device__ __forceinline__ float2 exp2_poly2(float2 y)
+{
+    y = make_float2(fmaxf(y.x, -125.f), fmaxf(y.y, -125.f));
+    const float2 t = __fadd2_rn(y, make_float2(kRoundMagic, kRoundMagic));
+    const float2 n = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));
+    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), y);
+    float2 q = __ffma2_rn(make_float2(kP3, kP3), f, make_float2(kP2, kP2));
+    q = __ffma2_rn(q, f, make_float2(kP1, kP1));
+    q = __ffma2_rn(q, f, make_float2(kP0, kP0));
+    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// Key-validity mask of one 32-column chunk: x = -inf where key0 + e lies
+// outside [lo, hi].
+__device__ __forceinline__ void mask_chunk(float (&x)[32], int key0, int lo, int hi)
+{
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int key = key0 + e;
+        if (key < lo || key > hi) x[e] = -INFINITY;
+    }
+}
+
+__device__ __forceinline__ float chunk_max(const float (&x)[32])
+{
+    float m[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) m[i] = fmax3(x[8 * i], x[8 * i + 1], x[8 * i + 2]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        m[i] = fmax3(m[i], x[8 * i + 3], x[8 * i + 4]);
+        m[i] = fmax3(m[i], x[8 * i + 5], x[8 * i + 6]);
+        m[i] = fmaxf(m[i], x[8 * i + 7]);
+    }
+    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
+}
+
+__device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
+{
+    uint32_t u[32];
+    tmem_ld32_wait(addr, u);
+#pragma unroll
+    for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(u[e]);
+}
+
+// 2^y for a pair on the MUFU unit in half precision: y is rounded to fp16
+// and one ex2.approx.f16x2 yields both exponentials as the fp16 pair the
+// P V MMA consumes (y <= 8 here; an fp16 y keeps the error of 2^y below a
+// few fp16 spacings of the result).
+__device__ __forceinline__ uint32_t exp2_f16x2(float y0, float y1)
+{
+    uint32_t h, e;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(y1), "f"(y0));
+    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
+    return e;
+}
+
+// acc + (fp16 value), exact widening of the fp16 operand.
+__device__ __forceinline__ float add_f16(float acc, uint16_t h)
+{
+    float d;
+    asm("{.reg .f16 t; mov.b16 t, %1; add.rn.f32.f16 %0, t, %2;}" : "=f"(d) : "h"(h), "f"(acc));
+    return d;
+}
+
+// Softmax numerators of one 32-column chunk: p = 2^(x c - m), packed to
+// 16-bit pairs (fp16 for core tiles, bf16 for raw ones) and stored to tensor
+// memory at p_addr (16 columns).  The MUFU unit computes 16 exponentials
+// per clock per SM, as many as the tile's MMAs need at full rate, so pairs
+// i with (i % 8) < kPolyPerEight take the FMA-pipe polynomial instead.  The
+// row sum is accumulated in acc from exactly the 16-bit values P V will see,
+// so that the rounding of a dominant weight cancels in O = (P V) / l.
+template <bool F16>
+__device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float2 nm2,
+                                          uint32_t p_addr, float2 &acc)
+{
+    uint32_t pk[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const float2 y = __ffma2_rn(make_float2(x[2 * i], x[2 * i + 1]), c2, nm2);
+        if ((i & 7) < kPolyPerEight) {
+            const float2 pv = exp2_poly2(y);
+            pk[i] = F16 ? pack_f16x2(pv.x, pv.y) : pack_bf16x2(pv.x, pv.y);
+        } else if (F16) {
+            pk[i] = exp2_f16x2(y.x, y.y);
+        } else {
+            pk[i] = pack_bf16x2(fast_exp2(y.x), fast_exp2(y.y));
+        }
+        if (F16) {
+            acc.x = add_f16(acc.x, static_cast<uint16_t>(pk[i] & 0xFFFFu));
+            acc.y = add_f16(acc.y, static_cast<uint16_t>(pk[i] >> 16));
+        } else {
+            acc = __fadd2_rn(acc, make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
+        }
+    }
+    tmem_st16(p_addr, pk);
+}
+
+__device__ __forceinline__ float row_max128(const float (&x)[128])
+{
+    float m[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmax3(x[16 * i], x[16 * i + 1], x[16 * i + 2]);
+#pragma unroll
+    for (int k = 3; k < 15; k += 2)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m[i] = fmax3(m[i], x[16 * i + k], x[16 * i + k + 1]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], x[16 * i + 15]);
+    return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV,
@@ -159,7 +304,6 @@ __global__ void __launch_bounds__(192, 1)
     uint8_t *smem = reinterpret_cast<uint8_t *>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sQ = smem + C::OFF_Q;
-    uint8_t *sQh = smem + C::OFF_QH;
     uint8_t *sK = smem + C::OFF_K;
     uint8_t *sV = smem + C::OFF_V;
     Bars *bars = reinterpret_cast<Bars *>(smem + C::OFF_BAR);
@@ -169,7 +313,7 @@ __global__ void __launch_bounds__(192, 1)
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
-        mbar_init(&bars->qh_full, 4);
+        mbar_init(&bars->qloc_done, 1);
         for (int s = 0; s < C::KST; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
@@ -178,18 +322,19 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&bars->v_full[s], 1);
             mbar_init(&bars->v_empty[s], 1);
         }
-        for (int b = 0; b < 2; ++b) {
-            mbar_init(&bars->s_full[b], 1);
-            mbar_init(&bars->p_full[b], 4);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bars->qh_full[h], 4);
+            mbar_init(&bars->s_full[h], 1);
+            mbar_init(&bars->p_full[h], 4);
+            mbar_init(&bars->o_bar[h], 1);
+            mbar_init(&bars->o_empty[h], 4);
         }
-        mbar_init(&bars->o_bar, 1);
-        mbar_init(&bars->o_empty, 4);
         mbar_init(&bars->mma_done, 1);
         bars->abort = 0;
         bars->never = 0;
         mbar_fence_init();
     }
-    if (warp == 4) {
+    if (warp == 8) {
         tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
         tmem_relinquish();
         if (lane == 0) {
@@ -205,7 +350,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
+    if (warp == 8) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t kc = 0, vc = 0, qc = 0;
@@ -213,10 +358,12 @@ __global__ void __launch_bounds__(192, 1)
             for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
                 const Geom G = geom(item, p);
                 if (qc > 0 && !(ok = lane_wait(&bars->q_empty, (qc - 1) & 1, bars))) break;
-                mbar_arrive_expect_tx(&bars->q_full, C::TILE_BYTES);
-                for (int bx = 0; bx < C::NBOX; ++bx)
-                    tma_load_3d(sQ + bx * C::BOX_BYTES, &tmQ, &bars->q_full, bx * 64,
-                                G.t0, G.b * p.Hq + G.hq);
+                mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
+                for (int hh = 0; hh < 2; ++hh)
+                    for (int bx = 0; bx < C::NBOX; ++bx)
+                        tma_load_3d(sQ + hh * C::TILE_BYTES + bx * C::BOX_BYTES, &tmQ,
+                                    &bars->q_full, bx * 64, G.t0 + hh * 128,
+                                    G.b * p.Hq + G.hq);
                 ++qc;
                 const int z = G.b * p.Hkv + G.h;
                 for (int j = 0; j < G.n_tiles; ++j) {
@@ -247,7 +394,7 @@ __global__ void __launch_bounds__(192, 1)
                 }
             }
             // Drain: every issued copy must have landed before the CTA exits
-            // (the last fill of each ring stage, and the last Q tile).
+            // (the last fill of each ring stage, and the last Q block).
             const volatile int *never = &bars->never;
             for (uint32_t s = 0; s < C::KST && s < kc; ++s) {
                 const uint32_t last = kc - 1 - ((kc - 1 - s) % C::KST);
@@ -261,142 +408,143 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (qc > 0) wait_bounded(&bars->q_full, (qc - 1) & 1, never, kWaitLimitNs);
         }
-    } else if (warp == 5) {
+    } else if (warp == 9) {
         // ------------------------------------------------ tcgen05 issuer
         if (lane == 0) {
             constexpr uint32_t idesc_qk_bf = idesc_f32acc(128, 128, true, false, false);
             constexpr uint32_t idesc_qk_h = idesc_f32acc(128, 128, false, false, false);
             constexpr uint32_t idesc_pv_bf = idesc_f32acc(128, D, true, false, true);
             constexpr uint32_t idesc_pv_h = idesc_f32acc(128, D, false, false, true);
-            const uint32_t q_base = smem_addr(sQ), qh_base = smem_addr(sQh),
-                           k_base = smem_addr(sK), v_base = smem_addr(sV);
-            uint32_t kc = 0, vc = 0, it = 0, qhc = 0;
+            const uint32_t q_base = smem_addr(sQ), k_base = smem_addr(sK),
+                           v_base = smem_addr(sV);
+            uint32_t kc = 0, vc = 0, it = 0, cq = 0;
             int k = 0;
             bool ok = true;
+            // Shared-memory descriptors: the start-address field (bits
+            // 0-13, 16-byte units) is advanced by plain addition.
+            const uint64_t dq = smem_desc_sw128(q_base, 16, 1024);
+            const uint64_t dk = smem_desc_sw128(k_base, 16, 1024);
+            const uint64_t dv = smem_desc_sw128(v_base, C::BOX_BYTES, 1024);
+            constexpr uint32_t kTile16 = C::TILE_BYTES >> 4;
+            auto qk = [&](int hh, uint32_t s, bool core) {
+                const uint64_t a0 = dq + hh * kTile16, b0 = dk + s * kTile16;
+                const uint32_t idesc = core ? idesc_qk_h : idesc_qk_bf;
+                const uint32_t d_tmem = tmem + C::S_COL + hh * 128;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    constexpr uint32_t box16 = C::BOX_BYTES >> 4;
+                    const uint32_t off = (kk >> 2) * box16 + (kk & 3) * 2;
+                    mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+                }
+            };
+            auto pv = [&](int hh, uint32_t sv, bool core, bool first) {
+                const uint64_t b0 = dv + sv * kTile16;
+                const uint32_t idesc = core ? idesc_pv_h : idesc_pv_bf;
+                const uint32_t d_tmem = tmem + C::O_COL + hh * D;
+                const uint32_t a_tmem = tmem + C::S_COL + hh * 128;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc,
+                           (first && kk == 0) ? 0u : 1u);
+            };
             for (int item = blockIdx.x; ok && item < p.n_items;
                  item += gridDim.x, ++k) {
                 const Geom G = geom(item, p);
+                const bool core_block = G.n_core_tiles > 0;
                 if (!(ok = lane_wait(&bars->q_full, k & 1, bars))) break;
                 const uint32_t it0 = it;
-                auto issue_pv = [&](int jj) -> bool {
+                // P V of tile jj for half hh (V stage waited by half A).
+                auto issue_pv = [&](int hh, int jj) -> bool {
                     const uint32_t itp = it0 + jj;
-                    const uint32_t bp = itp & 1;
-                    if (!lane_wait(&bars->p_full[bp], (itp >> 1) & 1, bars)) return false;
+                    if (!lane_wait(&bars->p_full[hh], itp & 1, bars)) return false;
+                    if (jj == 0 && k > 0 && !lane_wait(&bars->o_empty[hh], (k - 1) & 1, bars))
+                        return false;
                     const uint32_t sv = vc % C::VST;
-                    if (!lane_wait(&bars->v_full[sv], (vc / C::VST) & 1, bars)) return false;
-                    if (jj == 0 && k > 0 && !lane_wait(&bars->o_empty, (k - 1) & 1, bars))
+                    if (hh == 0 && !lane_wait(&bars->v_full[sv], (vc / C::VST) & 1, bars))
                         return false;
                     tc_fence_after_sync();
-                    const uint32_t idesc = tile_is_core(G, jj) ? idesc_pv_h : idesc_pv_bf;
-                    const uint32_t vs = v_base + sv * C::TILE_BYTES;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const uint64_t bdesc =
-                            smem_desc_sw128(vs + kk * 16 * 128, C::BOX_BYTES, 1024);
-                        mma_ts(tmem + C::O_COL, tmem + bp * C::S_STRIDE + kk * 8, bdesc,
-                               idesc, (jj > 0 || kk > 0) ? 1u : 0u);
+                    pv(hh, sv, tile_is_core(G, jj), jj == 0);
+                    mma_commit(&bars->o_bar[hh]);
+                    if (hh == 1) {
+                        mma_commit(&bars->v_empty[sv]);
+                        ++vc;
                     }
-                    mma_commit(&bars->o_bar);
-                    mma_commit(&bars->v_empty[sv]);
-                    ++vc;
                     return true;
                 };
-                for (int j = 0; j < G.n_tiles; ++j) {
-                    const uint32_t b = it & 1;
+                for (int j = 0; ok && j < G.n_tiles; ++j) {
                     const bool core = tile_is_core(G, j);
-                    if (core && j == G.n_local) {
-                        // the fp16 copy of Q is written by the softmax warps
-                        if (!(ok = lane_wait(&bars->qh_full, qhc & 1, bars))) break;
-                        ++qhc;
-                    }
                     const uint32_t s = kc % C::KST;
                     if (!(ok = lane_wait(&bars->k_full[s], (kc / C::KST) & 1, bars))) break;
-                    tc_fence_after_sync();
-                    const uint32_t ks = k_base + s * C::TILE_BYTES;
-                    const uint32_t qs = core ? qh_base : q_base;
-                    const uint32_t idesc = core ? idesc_qk_h : idesc_qk_bf;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t off = (kk >> 2) * C::BOX_BYTES + (kk & 3) * 32;
-                        const uint64_t adesc = smem_desc_sw128(qs + off, 16, 1024);
-                        const uint64_t bdesc = smem_desc_sw128(ks + off, 16, 1024);
-                        mma_ss(tmem + b * C::S_STRIDE, adesc, bdesc, idesc, kk > 0 ? 1u : 0u);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (j > 0 && !(ok = issue_pv(hh, j - 1))) break;
+                        if (core && j == G.n_local &&
+                            !(ok = lane_wait(&bars->qh_full[hh], cq & 1, bars)))
+                            break;
+                        tc_fence_after_sync();
+                        qk(hh, s, core);
+                        mma_commit(&bars->s_full[hh]);
                     }
-                    mma_commit(&bars->s_full[b]);
+                    if (!ok) break;
                     mma_commit(&bars->k_empty[s]);
                     ++kc;
-                    if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
                     ++it;
-                    if (j > 0 && !(ok = issue_pv(j - 1))) break;
+                    if (core_block && j == G.n_local - 1) mma_commit(&bars->qloc_done);
+                    if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
                 }
-                if (ok) ok = issue_pv(G.n_tiles - 1);
+                if (ok) ok = issue_pv(0, G.n_tiles - 1) && issue_pv(1, G.n_tiles - 1);
+                if (core_block) ++cq;
             }
             // Wait for every issued tensor-core operation to finish.
             mma_commit(&bars->mma_done);
             wait_bounded(&bars->mma_done, 0, &bars->never, kWaitLimitNs);
         }
-    } else {
+    } else if (warp < 8) {
         // ------------------------------------------------ softmax warps
-        const int row = threadIdx.x;  // 0..127 = tensor-memory lane
-        const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-        uint32_t it = 0, pv_waits = 0, k = 0;
+        const int hh = warp >> 2;                  // half
+        const int row = threadIdx.x & 127;         // tensor-memory lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t s_addr = tmem + lane_off + C::S_COL + hh * 128;
+        const uint32_t o_addr = tmem + lane_off + C::O_COL + hh * D;
+        uint32_t it = 0, pv_waits = 0, cq = 0;
         bool ok = true;
-        for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x, ++k) {
+        for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
             const Geom G = geom(item, p);
-            const int t = G.t0 + row;
+            const bool core_block = G.n_core_tiles > 0;
+            const int t0h = G.t0 + hh * 128;       // first row of this half
+            const int t = t0h + row;
             const int ws_t = ws_of(t, p.g, p.w);
             const int nc_t = ws_t / p.g;
-            if (!(ok = warp_wait(&bars->q_full, k & 1, bars))) break;
-            if (G.n_core_tiles > 0) {
-                // fp16 copy of the Q tile for the core stream (same swizzled
-                // layout: 16-byte chunks of 8 elements keep their places)
-                bool over = false;
-                const uint4 *src = reinterpret_cast<const uint4 *>(sQ);
-                uint4 *dst = reinterpret_cast<uint4 *>(sQh);
-#pragma unroll 4
-                for (int c = threadIdx.x; c < C::TILE_BYTES / 16; c += 128) {
-                    const uint4 v = src[c];
-                    uint4 h;
-                    h.x = pack_f16x2(clamp_f16(bf16_lo(v.x), over), clamp_f16(bf16_hi(v.x), over));
-                    h.y = pack_f16x2(clamp_f16(bf16_lo(v.y), over), clamp_f16(bf16_hi(v.y), over));
-                    h.z = pack_f16x2(clamp_f16(bf16_lo(v.z), over), clamp_f16(bf16_hi(v.z), over));
-                    h.w = pack_f16x2(clamp_f16(bf16_lo(v.w), over), clamp_f16(bf16_hi(v.w), over));
-                    dst[c] = h;
-                }
-                if (over) atomicOr(&g_prefill_status, kStatusRange);
-                fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->qh_full);
-            }
+            const int nc_lo = ws_of(t0h, p.g, p.w) / p.g;
+            const int ws_hi = ws_of(t0h + 127, p.g, p.w);
             float m_run = -INFINITY, l_run = 0.f;
             for (int j = 0; j < G.n_tiles; ++j, ++it) {
-                const uint32_t b = it & 1;
-                if (!(ok = warp_wait(&bars->s_full[b], (it >> 1) & 1, bars))) break;
+                if (!(ok = warp_wait(&bars->s_full[hh], it & 1, bars))) break;
                 tc_fence_after_sync();
-                float x[128];
-                {
-                    uint32_t u[128];
-                    tmem_ld128_wait(tmem + lane_off + b * C::S_STRIDE, u);
-#pragma unroll
-                    for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
-                }
-                // Mask keys this row does not see.
                 const bool core = tile_is_core(G, j);
                 const int key0 = tile_key0(G, j);
-                const bool need_mask = core ? (key0 + 128 > G.nc_lo)
-                                            : (key0 < G.ws_hi || key0 + 127 > G.t0);
-                if (need_mask) {
-                    const int lo = core ? 0 : ws_t;
-                    const int hi = core ? nc_t - 1 : t;
+                const bool need_mask = core ? (key0 + 128 > nc_lo)
+                                            : (key0 < ws_hi || key0 + 127 > t0h);
+                const int lo = core ? 0 : ws_t;
+                const int hi = core ? nc_t - 1 : t;
+                // pass 1: row maximum of the tile (one 128-column load)
+                float mx;
+                {
+                    float x[128];
+                    {
+                        uint32_t u[128];
+                        tmem_ld128_wait(s_addr, u);
 #pragma unroll
-                    for (int e = 0; e < 128; ++e) {
-                        const int key = key0 + e;
-                        if (key < lo || key > hi) x[e] = -INFINITY;
+                        for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
                     }
-                }
-                float mx = x[0];
+                    if (need_mask) {
 #pragma unroll
-                for (int e = 1; e < 128; ++e) mx = fmaxf(mx, x[e]);
+                        for (int e = 0; e < 128; ++e) {
+                            const int key = key0 + e;
+                            if (key < lo || key > hi) x[e] = -INFINITY;
+                        }
+                    }
+                    mx = row_max128(x);
+                }
                 const float m_tile = mx * p.scale_log2;
                 float alpha = 1.f;
                 if (m_tile > m_run + kRescaleThreshold) {
@@ -404,95 +552,113 @@ __global__ void __launch_bounds__(192, 1)
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                // P in the element type of this tile's values (fp16 core,
-                // bf16 raw); the row sum uses the rounded weights P V sees.
-                uint32_t pk[64];
-                float rs = 0.f;
-                if (core) {
+                // pass 2: P = 2^(S c - m) over the S columns already read
+                // (chunk c's 32 logits become 16 packed columns at c*16, below
+                // the chunks still to be read; the MMA reads P only after
+                // p_full below).
+                const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
+                const float2 nm2 = make_float2(-m_use, -m_use);
+                float2 acc = make_float2(0.f, 0.f);
+                // (the chunk loop stays rolled: unrolled, the softmax code
+                // outgrows the instruction cache and runs slower)
+#pragma unroll 1
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t u[32];
+                    tmem_ld32_wait(s_addr + c * 32, u);
+                    float x[32];
 #pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const float p0 = fast_exp2(fmaf(x[2 * e], p.scale_log2, -m_use));
-                        const float p1 = fast_exp2(fmaf(x[2 * e + 1], p.scale_log2, -m_use));
-                        pk[e] = pack_f16x2(p0, p1);
-                        rs += f16_lo(pk[e]) + f16_hi(pk[e]);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 64; ++e) {
-                        const float p0 = fast_exp2(fmaf(x[2 * e], p.scale_log2, -m_use));
-                        const float p1 = fast_exp2(fmaf(x[2 * e + 1], p.scale_log2, -m_use));
-                        pk[e] = pack_bf16x2(p0, p1);
-                        rs += bf16_lo(pk[e]) + bf16_hi(pk[e]);
-                    }
+                    for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(u[e]);
+                    if (need_mask) mask_chunk(x, key0 + c * 32, lo, hi);
+                    if (core)
+                        exp_chunk<true>(x, c2, nm2, s_addr + c * 16, acc);
+                    else
+                        exp_chunk<false>(x, c2, nm2, s_addr + c * 16, acc);
                 }
+                const float rs = acc.x + acc.y;
                 l_run = fmaf(l_run, alpha, rs);
                 if (j > 0) {
-                    // O must hold P V of the previous tile before it is rescaled
-                    if (!(ok = warp_wait(&bars->o_bar, pv_waits & 1, bars))) break;
+                    // P V of the previous tile is complete (it was issued
+                    // before this tile's S); rescale O if the max moved
+                    if (!(ok = warp_wait(&bars->o_bar[hh], pv_waits & 1, bars))) break;
                     ++pv_waits;
                     tc_fence_after_sync();
                     if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
                         for (int c = 0; c < D / 32; ++c) {
                             uint32_t u[32];
-                            tmem_ld32_wait(tmem + lane_off + C::O_COL + c * 32, u);
+                            tmem_ld32_wait(o_addr + c * 32, u);
 #pragma unroll
                             for (int e = 0; e < 32; ++e)
                                 u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-                            tmem_st32(tmem + lane_off + C::O_COL + c * 32, u);
+                            tmem_st32(o_addr + c * 32, u);
                         }
                     }
-                }
-                {
-                    uint32_t u[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] = pk[e];
-                    tmem_st32(tmem + lane_off + b * C::S_STRIDE, u);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] = pk[32 + e];
-                    tmem_st32(tmem + lane_off + b * C::S_STRIDE + 32, u);
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full[b]);
+                if (lane == 0) mbar_arrive(&bars->p_full[hh]);
+                if (core_block && j == G.n_local - 1) {
+                    // Last local tile done: once every local Q K^T has read
+                    // the bf16 Q block, turn this half into fp16 in place for
+                    // the core stream (16-byte chunks of 8 elements keep
+                    // their swizzled places).
+                    if (!(ok = warp_wait(&bars->qloc_done, cq & 1, bars))) break;
+                    bool over = false;
+                    uint4 *q4 = reinterpret_cast<uint4 *>(sQ + hh * C::TILE_BYTES);
+#pragma unroll 4
+                    for (int c = row; c < C::TILE_BYTES / 16; c += 128) {
+                        const uint4 v = q4[c];
+                        uint4 h;
+                        h.x = pack_f16x2(clamp_f16(bf16_lo(v.x), over), clamp_f16(bf16_hi(v.x), over));
+                        h.y = pack_f16x2(clamp_f16(bf16_lo(v.y), over), clamp_f16(bf16_hi(v.y), over));
+                        h.z = pack_f16x2(clamp_f16(bf16_lo(v.z), over), clamp_f16(bf16_hi(v.z), over));
+                        h.w = pack_f16x2(clamp_f16(bf16_lo(v.w), over), clamp_f16(bf16_hi(v.w), over));
+                        q4[c] = h;
+                    }
+                    if (over) atomicOr(&g_prefill_status, kStatusRange);
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->qh_full[hh]);
+                }
             }
             if (!ok) break;
+            if (core_block) ++cq;
             // Epilogue: O / l for this row.
-            if (!(ok = warp_wait(&bars->o_bar, pv_waits & 1, bars))) break;
+            if (!(ok = warp_wait(&bars->o_bar[hh], pv_waits & 1, bars))) break;
             ++pv_waits;
             tc_fence_after_sync();
-            float o[D];
+            // O / l for this row, 32 columns at a time; O is read completely
+            // before its tensor memory is released
+            const float inv = 1.0f / l_run;
+            const int64_t orow = (static_cast<int64_t>(G.b) * p.Hq + G.hq) * p.T + t;
+            const bool store = t < p.T;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
-                uint32_t u[32];
-                tmem_ld32_wait(tmem + lane_off + C::O_COL + c * 32, u);
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o[c * 32 + e] = __uint_as_float(u[e]);
-            }
-            tc_fence_before_sync();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&bars->o_empty);
-            if (t < p.T) {
-                const float inv = 1.0f / l_run;
-                const int64_t orow =
-                    (static_cast<int64_t>(G.b) * p.Hq + G.hq) * p.T + t;
+                float o[32];
+                load_chunk(o_addr + c * 32, o);
+                if (c == D / 32 - 1) {
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->o_empty[hh]);
+                }
+                if (!store) continue;
                 if (p.o_f32) {
                     float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(p.O) +
-                                                             orow * D);
+                                                             orow * D + c * 32);
 #pragma unroll
-                    for (int c = 0; c < D / 4; ++c)
-                        dst[c] = make_float4(o[4 * c] * inv, o[4 * c + 1] * inv,
-                                             o[4 * c + 2] * inv, o[4 * c + 3] * inv);
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(o[4 * q] * inv, o[4 * q + 1] * inv,
+                                             o[4 * q + 2] * inv, o[4 * q + 3] * inv);
                 } else {
                     uint4 *dst = reinterpret_cast<uint4 *>(static_cast<uint16_t *>(p.O) +
-                                                           orow * D);
+                                                           orow * D + c * 32);
 #pragma unroll
-                    for (int c = 0; c < D / 8; ++c)
-                        dst[c] = make_uint4(pack_bf16x2(o[8 * c] * inv, o[8 * c + 1] * inv),
-                                            pack_bf16x2(o[8 * c + 2] * inv, o[8 * c + 3] * inv),
-                                            pack_bf16x2(o[8 * c + 4] * inv, o[8 * c + 5] * inv),
-                                            pack_bf16x2(o[8 * c + 6] * inv, o[8 * c + 7] * inv));
+                    for (int q = 0; q < 4; ++q)
+                        dst[q] = make_uint4(pack_bf16x2(o[8 * q] * inv, o[8 * q + 1] * inv),
+                                            pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv),
+                                            pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv),
+                                            pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv));
                 }
             }
         }
@@ -500,7 +666,7 @@ __global__ void __launch_bounds__(192, 1)
 
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == 8) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, C::TMEM_COLS);
     }
@@ -570,8 +736,8 @@ cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc
     p.g = g;
     p.w = w;
     p.m = static_cast<int>(m);
-    p.n_qtiles = static_cast<int>((T + 127) / 128);
-    p.n_items = p.n_qtiles * B * Hq;
+    p.n_blocks = static_cast<int>((T + 255) / 256);
+    p.n_items = p.n_blocks * B * Hq;
     p.scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
     p.O = O;
     p.o_f32 = o_f32 ? 1 : 0;
@@ -582,7 +748,7 @@ cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc
     cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    prefill_kernel<D><<<grid, 192, C::SMEM, s>>>(mQ, mK, mV, mKc, mVc, p);
+    prefill_kernel<D><<<grid, C::THREADS, C::SMEM, s>>>(mQ, mK, mV, mKc, mVc, p);
     return cudaGetLastError();
 }
 

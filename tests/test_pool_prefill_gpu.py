@@ -24,6 +24,8 @@ CASES = [
     (1, 2, 2, 1000, 128, 4, 50),    # core stream spans two key tiles
     (1, 2, 2, 517, 128, 5, 37),     # g not dividing w or T
     (1, 3, 1, 700, 64, 32, 100),    # r = 3
+    (8, 16, 8, 384, 128, 16, 64),   # 384 work items: several per CTA, 1-4 tiles each
+    (4, 32, 8, 1100, 128, 32, 200), # grouped heads, many items with and without core
 ]
 
 
