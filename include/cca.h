@@ -68,7 +68,8 @@ typedef enum {
     CCA_ERR_CAPACITY = 3,    /* cache has no room for the request          */
     CCA_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed          */
     CCA_ERR_TIMEOUT = 5,     /* a bounded device-side wait ran out         */
-    CCA_ERR_RANGE = 6        /* a value beyond the fp16 range was clamped  */
+    CCA_ERR_RANGE = 6,       /* a value beyond the fp16 range was clamped  */
+    CCA_ERR_SCRATCH = 7      /* request exceeds the library's fixed scratch */
 } cca_status;
 
 /* Element type of an output that may be written in either precision. */
@@ -160,6 +161,30 @@ size_t cca_decode_workspace_bytes(const cca_cache *c);
 cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                            cca_dtype o_dtype, void *workspace,
                            size_t workspace_bytes, cudaStream_t stream);
+
+/* Size of the library's fixed decode scratch (bytes): the largest
+ * cca_decode_workspace_bytes() that cca_attn_decode_noalloc can serve. */
+#define CCA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/*
+ * cca_attn_decode without a caller-provided workspace.  The paper has no
+ * counterpart: this is a service for callers that cannot allocate device
+ * memory, such as runtimes that plan all device memory up front and forbid
+ * other allocations, plug-in hosts that only pass input and output pointers,
+ * or latency-critical loops that cannot afford cudaMalloc (which may
+ * synchronise the device).  It computes exactly what cca_attn_decode
+ * computes, with the split-K partials in a fixed array of
+ * CCA_NOALLOC_SCRATCH_BYTES that the library holds on every GPU it is loaded
+ * on until the process exits; it allocates nothing.
+ *   Returns CCA_ERR_SCRATCH (nothing launched) if the cache needs more
+ *   workspace than that array; other errors as cca_attn_decode.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current), so make it before any stream capture begins.
+ *   All calls share the array: calls whose kernels may overlap on the GPU
+ *   (e.g. on unordered streams) race.  Nothing in it needs clearing.
+ */
+cca_status cca_attn_decode_noalloc(const cca_cache *c, const void *q_t, void *o_t,
+                                   cca_dtype o_dtype, cudaStream_t stream);
 
 /*
  * Synchronise `stream`, then report CCA_ERR_CUDA if a CUDA error is

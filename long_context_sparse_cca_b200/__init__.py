@@ -30,13 +30,16 @@ CCA_ERR_CAPACITY = 3
 CCA_ERR_CUDA = 4
 CCA_ERR_TIMEOUT = 5
 CCA_ERR_RANGE = 6
+CCA_ERR_SCRATCH = 7
 CCA_BF16 = 0
 CCA_F32 = 1
+NOALLOC_SCRATCH_BYTES = 4 << 20  # CCA_NOALLOC_SCRATCH_BYTES of include/cca.h
 
 # Every symbol include/cca.h declares.
 EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
-           "cca_device_status", "cca_status_string", "cca_version", "cca_last_error")
+           "cca_device_status", "cca_status_string", "cca_version", "cca_last_error",
+           "cca_attn_decode_noalloc")
 
 
 class CCAError(RuntimeError):
@@ -83,6 +86,8 @@ def lib():
     L.cca_decode_workspace_bytes.restype = ctypes.c_size_t
     L.cca_attn_decode.argtypes = [CP, P, P, i, P, ctypes.c_size_t, P]
     L.cca_attn_decode.restype = st
+    L.cca_attn_decode_noalloc.argtypes = [CP, P, P, i, P]
+    L.cca_attn_decode_noalloc.restype = st
     L.cca_device_status.argtypes = [P]
     L.cca_device_status.restype = st
     L.cca_status_string.argtypes = [i]
@@ -272,6 +277,20 @@ def cca_attn_decode(cache: Cache, q_t, o_t=None, out_dtype=None,
         ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(o_t, "o_t", o_t.dtype),
         od, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
         _stream(stream)), "cca_attn_decode")
+    return o_t
+
+
+def cca_attn_decode_noalloc(cache: Cache, q_t, o_t=None, out_dtype=None, stream=None):
+    """As cca_attn_decode, with the library's fixed device scratch in place
+    of a workspace (for callers that cannot allocate device memory)."""
+    torch = _torch()
+    if o_t is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
+    od = _odtype(o_t.dtype)
+    _check(lib().cca_attn_decode_noalloc(
+        ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(o_t, "o_t", o_t.dtype), od,
+        _stream(stream)), "cca_attn_decode_noalloc")
     return o_t
 
 

@@ -210,6 +210,7 @@ const char *cca_status_string(cca_status s)
     case CCA_ERR_CUDA: return "CCA_ERR_CUDA";
     case CCA_ERR_TIMEOUT: return "CCA_ERR_TIMEOUT";
     case CCA_ERR_RANGE: return "CCA_ERR_RANGE";
+    case CCA_ERR_SCRATCH: return "CCA_ERR_SCRATCH";
     }
     return "CCA_ERR_UNKNOWN";
 }

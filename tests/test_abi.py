@@ -118,6 +118,27 @@ def test_cache_checks(L):
                              ws, None) == cca.CCA_ERR_INVALID_ARG  # dtype
 
 
+def test_noalloc_decode_refuses_oversized_cache(L):
+    """A cache whose decode workspace exceeds the library's fixed scratch is
+    refused before anything touches the GPU."""
+    P = ctypes.c_void_p
+    c = _cache(B=64, Hq=32, Hkv=32, core_cap=2048, length=100)
+    need = L.cca_decode_workspace_bytes(ctypes.byref(c))
+    assert need > cca.NOALLOC_SCRATCH_BYTES
+    st = L.cca_attn_decode_noalloc(ctypes.byref(c), P(FAKE), P(FAKE + 4096), 1, None)
+    assert st == cca.CCA_ERR_SCRATCH
+    assert cca.status_string(st) == "CCA_ERR_SCRATCH"
+    bad = _cache(tail_cap=10)  # invalid cache: the cache's own error
+    assert L.cca_attn_decode_noalloc(ctypes.byref(bad), P(FAKE), P(FAKE + 4096), 1,
+                                     None) == cca.CCA_ERR_INVALID_ARG
+
+
+def test_noalloc_scratch_size_matches_header():
+    with open(os.path.join(ROOT, "include", "cca.h")) as f:
+        m = re.search(r"#define CCA_NOALLOC_SCRATCH_BYTES \((\d+)u << (\d+)\)", f.read())
+    assert m and int(m.group(1)) << int(m.group(2)) == cca.NOALLOC_SCRATCH_BYTES
+
+
 def test_workspace_grows_with_capacity(L):
     a = _cache(core_cap=8)
     b = _cache(core_cap=4096)
