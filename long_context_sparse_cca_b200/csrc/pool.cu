@@ -13,8 +13,9 @@ namespace {
 
 constexpr int kPoolWarps = 8;  // warps per block
 
-template <int D>
-__global__ void __launch_bounds__(kPoolWarps * 32)
+// G > 0: register-resident fast path for that group size; G == 0: any g.
+template <int D, int G>
+__global__ void __launch_bounds__(kPoolWarps * 32, 2)
     pool_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                 const uint16_t *__restrict__ V, uint16_t *__restrict__ Kc,
                 uint16_t *__restrict__ Vc, int Hq, int Hkv, int64_t T, int g,
@@ -34,12 +35,18 @@ __global__ void __launch_bounds__(kPoolWarps * 32)
         const uint16_t *Vg = V + (bh * T + j * g) * D;
         const int64_t last = j * g + g - 1;
         const uint16_t *Qb = Q + ((b * Hq + h * r) * T + last) * D;
-        const bool over = pool_group_warp<D>(
-            [&](int i) { return Kg + static_cast<int64_t>(i) * D; },
-            [&](int i) { return Vg + static_cast<int64_t>(i) * D; },
-            [&](int k) { return Qb + static_cast<int64_t>(k) * T * D; }, r, g,
-            scale_log2, scratch, Kc + (bh * out_rows + j) * D,
-            Vc + (bh * out_rows + j) * D);
+        auto krow = [&](int i) { return Kg + static_cast<int64_t>(i) * D; };
+        auto vrow = [&](int i) { return Vg + static_cast<int64_t>(i) * D; };
+        auto qrow = [&](int k) { return Qb + static_cast<int64_t>(k) * T * D; };
+        bool over;
+        if constexpr (G > 0)
+            over = pool_group_warp_fast<D, G>(krow, vrow, qrow, r, scale_log2, scratch,
+                                              Kc + (bh * out_rows + j) * D,
+                                              Vc + (bh * out_rows + j) * D);
+        else
+            over = pool_group_warp<D>(krow, vrow, qrow, r, g, scale_log2, scratch,
+                                      Kc + (bh * out_rows + j) * D,
+                                      Vc + (bh * out_rows + j) * D);
         if (over && (threadIdx.x & 31) == 0) atomicOr(&g_pool_status, kStatusRange);
     }
 }
@@ -66,20 +73,27 @@ cudaError_t launch_pool(const void *Q, const void *K, const void *V, void *Kc,
     const auto *v = static_cast<const uint16_t *>(V);
     auto *kc = static_cast<uint16_t *>(Kc);
     auto *vc = static_cast<uint16_t *>(Vc);
+    auto go = [&](auto kern) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        kern<<<blocks, kPoolWarps * 32, smem, s>>>(q, k, v, kc, vc, Hq, Hkv, T, g, m,
+                                                    out_rows, n_groups, scale_log2);
+    };
     if (d == 128) {
-        if (smem > 48 * 1024)
-            cudaFuncSetAttribute(pool_kernel<128>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        pool_kernel<128><<<blocks, kPoolWarps * 32, smem, s>>>(
-            q, k, v, kc, vc, Hq, Hkv, T, g, m, out_rows, n_groups, scale_log2);
+        if (g == 16)
+            go(pool_kernel<128, 16>);
+        else if (g == 32)
+            go(pool_kernel<128, 32>);
+        else
+            go(pool_kernel<128, 0>);
     } else {
-        if (smem > 48 * 1024)
-            cudaFuncSetAttribute(pool_kernel<64>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-        pool_kernel<64><<<blocks, kPoolWarps * 32, smem, s>>>(
-            q, k, v, kc, vc, Hq, Hkv, T, g, m, out_rows, n_groups, scale_log2);
+        if (g == 16)
+            go(pool_kernel<64, 16>);
+        else if (g == 32)
+            go(pool_kernel<64, 32>);
+        else
+            go(pool_kernel<64, 0>);
     }
     return cudaGetLastError();
 }

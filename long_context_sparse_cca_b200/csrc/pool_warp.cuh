@@ -149,4 +149,130 @@ __device__ __forceinline__ bool pool_group_warp(KeyRow key_row, ValRow val_row,
     return __any_sync(0xffffffffu, over);
 }
 
+// ---------------------------------------------------------------------------
+// Register-resident pooling for a compile-time group size G (16 or 32).
+//
+// The warp is cut into RPW = 32 / (D/8) row slots of D/8 lanes; lane l owns
+// dims [8*(l % (D/8)), +8) of rows i with i % RPW == l / (D/8), loaded as
+// 16-byte vectors.  All of the group's key rows are requested before any
+// arithmetic (then all its value rows, for G = 32 only once the keys are
+// pooled), so each warp keeps G * 2 * D bytes in flight.  Scores are reduced
+// over the lanes of a row; the pooled sums are reduced over the row slots.
+// Same arithmetic as pool_group_warp: fp32 scores, fp32 softmax per query
+// head, mean over heads, fp32 weighted sums, fp16 stores.
+template <int D, int G, class KeyRow, class ValRow, class QRow>
+__device__ __forceinline__ bool pool_group_warp_fast(KeyRow key_row, ValRow val_row,
+                                                     QRow q_row, int r,
+                                                     float scale_log2, float *scratch,
+                                                     uint16_t *kc_out, uint16_t *vc_out)
+{
+    constexpr int LPR = D / 8;          // lanes per row
+    constexpr int RPW = 32 / LPR;       // rows per warp step
+    constexpr int NR = G / RPW;         // rows per lane
+    const int lane = threadIdx.x & 31;
+    const int kl = lane % LPR, slot = lane / LPR;
+    float *logit = scratch;             // [r][G]
+    float *weight = scratch + r * G;    // [G]
+
+    auto to8 = [](uint4 v, float (&f)[8]) {
+        f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+        f[4] = bf16_lo(v.z); f[5] = bf16_hi(v.z); f[6] = bf16_lo(v.w); f[7] = bf16_hi(v.w);
+    };
+    uint4 kv[NR], vv[NR];
+#pragma unroll
+    for (int n = 0; n < NR; ++n)
+        kv[n] = *reinterpret_cast<const uint4 *>(key_row(n * RPW + slot) + kl * 8);
+    if (G <= 16) {
+#pragma unroll
+        for (int n = 0; n < NR; ++n)
+            vv[n] = *reinterpret_cast<const uint4 *>(val_row(n * RPW + slot) + kl * 8);
+    }
+    // scores, all r query heads per key row
+    for (int k = 0; k < r; ++k) {
+        float q[8];
+        to8(*reinterpret_cast<const uint4 *>(q_row(k) + kl * 8), q);
+#pragma unroll
+        for (int n = 0; n < NR; ++n) {
+            float kf[8];
+            to8(kv[n], kf);
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) s = fmaf(q[e], kf[e], s);
+#pragma unroll
+            for (int o = 1; o < LPR; o <<= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+            if (kl == 0) logit[k * G + n * RPW + slot] = s * scale_log2;
+        }
+    }
+    __syncwarp();
+    // weights: mean over the r query heads of softmax over the G scores
+    if (lane < G) weight[lane] = 0.f;
+    if (G > 32) for (int i = lane + 32; i < G; i += 32) weight[i] = 0.f;
+    __syncwarp();
+    const float inv_r = 1.0f / static_cast<float>(r);
+    for (int k = 0; k < r; ++k) {
+        float mx = -INFINITY;
+        for (int i = lane; i < G; i += 32) mx = fmaxf(mx, logit[k * G + i]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int i = lane; i < G; i += 32) {
+            const float e = exp2f(logit[k * G + i] - mx);
+            logit[k * G + i] = e;
+            sum += e;
+        }
+        sum = warp_sum(sum);
+        const float c = inv_r / sum;
+        for (int i = lane; i < G; i += 32) weight[i] += logit[k * G + i] * c;
+    }
+    __syncwarp();
+    // pooled key, then pooled value
+    float ak[8], av[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ak[e] = av[e] = 0.f;
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+        const float a = weight[n * RPW + slot];
+        float kf[8];
+        to8(kv[n], kf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ak[e] = fmaf(a, kf[e], ak[e]);
+    }
+    if (G > 16) {
+#pragma unroll
+        for (int n = 0; n < NR; ++n)
+            vv[n] = *reinterpret_cast<const uint4 *>(val_row(n * RPW + slot) + kl * 8);
+    }
+#pragma unroll
+    for (int n = 0; n < NR; ++n) {
+        const float a = weight[n * RPW + slot];
+        float vf[8];
+        to8(vv[n], vf);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) av[e] = fmaf(a, vf[e], av[e]);
+    }
+#pragma unroll
+    for (int o = LPR; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], o);
+            av[e] += __shfl_xor_sync(0xffffffffu, av[e], o);
+        }
+    bool over = false;
+    if (slot == 0) {
+        uint4 h;
+        h.x = pack_f16x2(clamp_f16(ak[0], over), clamp_f16(ak[1], over));
+        h.y = pack_f16x2(clamp_f16(ak[2], over), clamp_f16(ak[3], over));
+        h.z = pack_f16x2(clamp_f16(ak[4], over), clamp_f16(ak[5], over));
+        h.w = pack_f16x2(clamp_f16(ak[6], over), clamp_f16(ak[7], over));
+        *reinterpret_cast<uint4 *>(kc_out + kl * 8) = h;
+    } else if (slot == 1) {
+        uint4 h;
+        h.x = pack_f16x2(clamp_f16(av[0], over), clamp_f16(av[1], over));
+        h.y = pack_f16x2(clamp_f16(av[2], over), clamp_f16(av[3], over));
+        h.z = pack_f16x2(clamp_f16(av[4], over), clamp_f16(av[5], over));
+        h.w = pack_f16x2(clamp_f16(av[6], over), clamp_f16(av[7], over));
+        *reinterpret_cast<uint4 *>(vc_out + kl * 8) = h;
+    }
+    return __any_sync(0xffffffffu, over);
+}
+
 }  // namespace cca
