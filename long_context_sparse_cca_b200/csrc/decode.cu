@@ -209,32 +209,56 @@ __global__ void __launch_bounds__(kDecodeThreads)
     }
 }
 
-// One warp per (batch, query head): combine the splits' partials.
+// One warp per (batch, query head): combine the splits' partials.  Lanes
+// take the splits in parallel for the maximum and the weights
+// 2^(m_s - max), which go to shared memory; then each lane adds its D/32
+// output dims over the splits with independent loads.
+constexpr int kMergeWarps = 4;
+
 template <int D>
-__global__ void decode_merge_kernel(const float *__restrict__ part_o,
-                                    const float2 *__restrict__ part_ml,
-                                    void *__restrict__ o_t, int out_f32,
-                                    int64_t rows, int nsplit)
+__global__ void __launch_bounds__(kMergeWarps * 32)
+    decode_merge_kernel(const float *__restrict__ part_o,
+                        const float2 *__restrict__ part_ml, void *__restrict__ o_t,
+                        int out_f32, int64_t rows, int nsplit)
 {
     constexpr int DPL = D / 32;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * (blockDim.x / 32) +
-                        (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
+    extern __shared__ float merge_w[];  // [kMergeWarps][nsplit]
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp;
     if (row >= rows) return;
+    float *w = merge_w + warp * nsplit;
+    const float2 *ml = part_ml + row * nsplit;
     float mx = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32) mx = fmaxf(mx, part_ml[row * nsplit + s].x);
+    for (int s = lane; s < nsplit; s += 32) mx = fmaxf(mx, ml[s].x);
     mx = warp_max(mx);
+    float l = 0.f;
+    for (int s = lane; s < nsplit; s += 32) {
+        const float2 v = ml[s];
+        const float c = fast_exp2(v.x - mx);
+        w[s] = c;
+        l = fmaf(c, v.y, l);
+    }
+    l = warp_sum(l);
+    __syncwarp();
     float acc[DPL];
 #pragma unroll
     for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    float l = 0.f;
+    const float *po = part_o + row * nsplit * D + lane * DPL;
+#pragma unroll 4
     for (int s = 0; s < nsplit; ++s) {
-        const float2 ml = part_ml[row * nsplit + s];
-        const float c = fast_exp2(ml.x - mx);
-        l = fmaf(c, ml.y, l);
-        const float *po = part_o + (row * nsplit + s) * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; ++e) acc[e] = fmaf(c, po[e], acc[e]);
+        const float c = w[s];
+        const float *src = po + static_cast<int64_t>(s) * D;
+        if constexpr (DPL == 4) {
+            const float4 v = *reinterpret_cast<const float4 *>(src);
+            acc[0] = fmaf(c, v.x, acc[0]);
+            acc[1] = fmaf(c, v.y, acc[1]);
+            acc[2] = fmaf(c, v.z, acc[2]);
+            acc[3] = fmaf(c, v.w, acc[3]);
+        } else {
+            const float2 v = *reinterpret_cast<const float2 *>(src);
+            acc[0] = fmaf(c, v.x, acc[0]);
+            acc[1] = fmaf(c, v.y, acc[1]);
+        }
     }
     const float inv = 1.0f / l;
     if (out_f32) {
@@ -342,16 +366,14 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
 #undef CCA_SPLIT
     if (e != cudaSuccess) return e;
     const int64_t rows = static_cast<int64_t>(B) * Hq;
-    const int wpb = 4;
-    const int blocks = static_cast<int>((rows + wpb - 1) / wpb);
+    const int blocks = static_cast<int>((rows + kMergeWarps - 1) / kMergeWarps);
+    const size_t msmem = sizeof(float) * kMergeWarps * p.nsplit;
     if (d == 128)
-        decode_merge_kernel<128><<<blocks, wpb * 32, 0, s>>>(part_o, part_ml, o_t,
-                                                             o_f32 ? 1 : 0, rows,
-                                                             p.nsplit);
+        decode_merge_kernel<128><<<blocks, kMergeWarps * 32, msmem, s>>>(
+            part_o, part_ml, o_t, o_f32 ? 1 : 0, rows, p.nsplit);
     else
-        decode_merge_kernel<64><<<blocks, wpb * 32, 0, s>>>(part_o, part_ml, o_t,
-                                                            o_f32 ? 1 : 0, rows,
-                                                            p.nsplit);
+        decode_merge_kernel<64><<<blocks, kMergeWarps * 32, msmem, s>>>(
+            part_o, part_ml, o_t, o_f32 ? 1 : 0, rows, p.nsplit);
     return cudaGetLastError();
 }
 

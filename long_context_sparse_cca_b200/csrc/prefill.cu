@@ -48,11 +48,18 @@ __device__ unsigned int g_prefill_status;  // kStatusTimeout | kStatusRange
 namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
-constexpr float kRescaleThreshold = 8.0f;         // log2 units: P stays <= 256
+constexpr float kRescaleThreshold = 15.0f;  // log2 units: P stays <= 2^15 (fp16 range)
+// Optionally the two halves take turns for the exponential passes of a
+// tile, so that their softmax phases do not share the MUFU unit.  Measured
+// on B200 at 128K context it is 8% slower (the softmax of one half is longer
+// than the other half's MMAs), so it is off.
+constexpr bool kTakeTurns = false;
 
 // Share of the exponentials computed on the FMA pipe: pairs i with
-// (i % 8) < kPolyPerEight of each 16-pair chunk of a row.
-constexpr int kPolyPerEight = 3;
+// (i % 8) < kPolyPerEight of each 16-pair chunk of a row.  Measured on B200
+// at 128K context: 0/8 14.3 ms, 2/8 14.6 ms, 3/8 15.2 ms (the polynomial's
+// extra issue slots cost more than the MUFU time it frees), so it is 0.
+constexpr int kPolyPerEight = 0;
 
 // 2^f on [-1/2, 1/2] by a degree-3 polynomial whose coefficients were fitted
 // for this kernel (Remez exchange on the relative error, weight 2^-f); max
@@ -136,6 +143,7 @@ struct Bars {
     uint64_t v_full[4], v_empty[4];
     uint64_t s_full[2], p_full[2];
     uint64_t o_bar[2], o_empty[2];
+    uint64_t turn[2];  // turn[h]: the other half finished its previous turn
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;  // set when any role gives up
@@ -224,33 +232,14 @@ __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
     for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(u[e]);
 }
 
-// 2^y for a pair on the MUFU unit in half precision: y is rounded to fp16
-// and one ex2.approx.f16x2 yields both exponentials as the fp16 pair the
-// P V MMA consumes (y <= 8 here; an fp16 y keeps the error of 2^y below a
-// few fp16 spacings of the result).
-__device__ __forceinline__ uint32_t exp2_f16x2(float y0, float y1)
-{
-    uint32_t h, e;
-    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(h) : "f"(y1), "f"(y0));
-    asm("ex2.approx.f16x2 %0, %1;" : "=r"(e) : "r"(h));
-    return e;
-}
-
-// acc + (fp16 value), exact widening of the fp16 operand.
-__device__ __forceinline__ float add_f16(float acc, uint16_t h)
-{
-    float d;
-    asm("{.reg .f16 t; mov.b16 t, %1; add.rn.f32.f16 %0, t, %2;}" : "=f"(d) : "h"(h), "f"(acc));
-    return d;
-}
-
 // Softmax numerators of one 32-column chunk: p = 2^(x c - m), packed to
 // 16-bit pairs (fp16 for core tiles, bf16 for raw ones) and stored to tensor
 // memory at p_addr (16 columns).  The MUFU unit computes 16 exponentials
 // per clock per SM, as many as the tile's MMAs need at full rate, so pairs
-// i with (i % 8) < kPolyPerEight take the FMA-pipe polynomial instead.  The
-// row sum is accumulated in acc from exactly the 16-bit values P V will see,
-// so that the rounding of a dominant weight cancels in O = (P V) / l.
+// i with (i % 8) < kPolyPerEight take the FMA-pipe polynomial instead.  For
+// bf16 P (8 significant bits) the row sum adds exactly the rounded values
+// P V will see, so that the rounding of a dominant weight cancels in
+// O = (P V) / l; for fp16 P (11 bits) the fp32 values are summed.
 template <bool F16>
 __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float2 nm2,
                                           uint32_t p_addr, float2 &acc)
@@ -259,18 +248,14 @@ __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float2 y = __ffma2_rn(make_float2(x[2 * i], x[2 * i + 1]), c2, nm2);
-        if ((i & 7) < kPolyPerEight) {
-            const float2 pv = exp2_poly2(y);
-            pk[i] = F16 ? pack_f16x2(pv.x, pv.y) : pack_bf16x2(pv.x, pv.y);
-        } else if (F16) {
-            pk[i] = exp2_f16x2(y.x, y.y);
-        } else {
-            pk[i] = pack_bf16x2(fast_exp2(y.x), fast_exp2(y.y));
-        }
+        const float2 pv = (i & 7) < kPolyPerEight
+                              ? exp2_poly2(y)
+                              : make_float2(fast_exp2(y.x), fast_exp2(y.y));
         if (F16) {
-            acc.x = add_f16(acc.x, static_cast<uint16_t>(pk[i] & 0xFFFFu));
-            acc.y = add_f16(acc.y, static_cast<uint16_t>(pk[i] >> 16));
+            pk[i] = pack_f16x2(pv.x, pv.y);
+            acc = __fadd2_rn(acc, pv);
         } else {
+            pk[i] = pack_bf16x2(pv.x, pv.y);
             acc = __fadd2_rn(acc, make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
         }
     }
@@ -328,6 +313,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&bars->p_full[h], 4);
             mbar_init(&bars->o_bar[h], 1);
             mbar_init(&bars->o_empty[h], 4);
+            mbar_init(&bars->turn[h], 4);
         }
         mbar_init(&bars->mma_done, 1);
         bars->abort = 0;
@@ -507,6 +493,7 @@ __global__ void __launch_bounds__(320, 1)
         const uint32_t o_addr = tmem + lane_off + C::O_COL + hh * D;
         uint32_t it = 0, pv_waits = 0, cq = 0;
         bool ok = true;
+        if (kTakeTurns && hh == 1 && lane == 0) mbar_arrive(&bars->turn[0]);  // A first
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
             const Geom G = geom(item, p);
             const bool core_block = G.n_core_tiles > 0;
@@ -526,6 +513,7 @@ __global__ void __launch_bounds__(320, 1)
                                             : (key0 < ws_hi || key0 + 127 > t0h);
                 const int lo = core ? 0 : ws_t;
                 const int hi = core ? nc_t - 1 : t;
+                if (kTakeTurns && !(ok = warp_wait(&bars->turn[hh], it & 1, bars))) break;
                 // pass 1: row maximum of the tile (one 128-column load)
                 float mx;
                 {
@@ -559,22 +547,44 @@ __global__ void __launch_bounds__(320, 1)
                 const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 acc = make_float2(0.f, 0.f);
-                // (the chunk loop stays rolled: unrolled, the softmax code
-                // outgrows the instruction cache and runs slower)
+                // Chunks are read in pairs, the second chunk's load in flight
+                // while the first is processed (a wait covers every earlier
+                // load, so the second load is issued after the first wait).
+                // The loop over the pairs stays rolled: fully unrolled, the
+                // softmax code outgrows the instruction cache.
 #pragma unroll 1
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t u[32];
-                    tmem_ld32_wait(s_addr + c * 32, u);
-                    float x[32];
+                for (int c = 0; c < 4; c += 2) {
+                    uint32_t ua[32], ub[32];
+                    tmem_ld32(s_addr + c * 32, ua);
+                    tmem_wait_ld_dep(ua);
+                    tmem_ld32(s_addr + (c + 1) * 32, ub);
+                    {
+                        float x[32];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(u[e]);
-                    if (need_mask) mask_chunk(x, key0 + c * 32, lo, hi);
-                    if (core)
-                        exp_chunk<true>(x, c2, nm2, s_addr + c * 16, acc);
-                    else
-                        exp_chunk<false>(x, c2, nm2, s_addr + c * 16, acc);
+                        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ua[e]);
+                        if (need_mask) mask_chunk(x, key0 + c * 32, lo, hi);
+                        if (core)
+                            exp_chunk<true>(x, c2, nm2, s_addr + c * 16, acc);
+                        else
+                            exp_chunk<false>(x, c2, nm2, s_addr + c * 16, acc);
+                    }
+                    tmem_wait_ld_dep(ub);
+                    {
+                        float x[32];
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ub[e]);
+                        if (need_mask) mask_chunk(x, key0 + (c + 1) * 32, lo, hi);
+                        if (core)
+                            exp_chunk<true>(x, c2, nm2, s_addr + (c + 1) * 16, acc);
+                        else
+                            exp_chunk<false>(x, c2, nm2, s_addr + (c + 1) * 16, acc);
+                    }
                 }
                 const float rs = acc.x + acc.y;
+                if (kTakeTurns) {
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bars->turn[hh ^ 1]);
+                }
                 l_run = fmaf(l_run, alpha, rs);
                 if (j > 0) {
                     // P V of the previous tile is complete (it was issued
