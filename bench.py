@@ -29,7 +29,9 @@ import argparse
 import json
 import os
 import statistics
+import shutil
 import subprocess
+import threading
 import sys
 import time
 
@@ -123,28 +125,44 @@ class ClockSampler:
         self.proc = None
 
     def __enter__(self):
-        self.first = ""
+        self.lines = []
+        self.proc = None
+        self.reader = None
+        cmd = ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
+               "--format=csv,noheader,nounits", "-lms", "100"]
+        # nvidia-smi block-buffers a pipe: line-buffer it so that samples
+        # arrive while the timed region runs, and read them on a thread
+        if shutil.which("stdbuf"):
+            cmd = ["stdbuf", "-oL"] + cmd
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu_index), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.proc = subprocess.Popen(cmd, stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
             # start timing only once the sampler is producing samples
-            self.first = self.proc.stdout.readline()
+            first = self.proc.stdout.readline()
+            if first:
+                self.lines.append(first)
+            self.reader = threading.Thread(target=self._read, daemon=True)
+            self.reader.start()
         except OSError:
             self.proc = None
         return self
 
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line)
+
     def __exit__(self, *exc):
-        self.out = ""
         if self.proc is not None:
+            time.sleep(0.15)  # one more sample of the end of the timed region
             self.proc.terminate()
             try:
-                self.out, _ = self.proc.communicate(timeout=5)
+                self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
-                self.out, _ = self.proc.communicate()
-            self.out = self.first + (self.out or "")
+                self.proc.wait()
+            if self.reader is not None:
+                self.reader.join(timeout=5)
+        self.out = "".join(self.lines)
         return False
 
     def summary(self) -> dict:

@@ -20,20 +20,24 @@
 // CTA of 320 threads (168 registers a thread: registers are booked for warps
 // in groups of four, so ten warps count as twelve):
 //   warps 0-3  softmax of half A, warps 4-7 softmax of half B: thread i owns
-//              query row i of its half; reads S from tensor memory, masks,
-//              online softmax (fp32; exp2 partly on the MUFU unit and partly
-//              as a polynomial on the FMA pipe; lazy rescale), writes P back
-//              into tensor memory over S, rescales O when its reference max
-//              moved, and runs the epilogue O / l.  At the switch from the
-//              local to the core stream each group turns its half of the Q
-//              tile from bf16 into fp16 in place.
+//              query row i of its half; copies its S row from tensor memory
+//              into registers (which frees S for the next Q K^T), masks,
+//              online softmax (fp32, exp2 on the MUFU unit, lazy rescale),
+//              writes P into its half's P buffer, rescales O when its
+//              reference max moved, and runs the epilogue O / l.  At the
+//              switch from the local to the core stream each group turns its
+//              half of the Q tile from bf16 into fp16 in place.
 //   warp 8     TMA producer: the Q block, then per key tile one K and one V
 //              tile into multi-stage shared-memory rings (128-byte swizzle).
-//   warp 9     tcgen05 issuer, ping-pong between the halves:
-//              ... O_A += P_A V_{j-1}; S_A = Q_A K_j^T; O_B += P_B V_{j-1};
-//              S_B = Q_B K_j^T ...  (S from shared memory operands, P from
-//              tensor memory).
-// Tensor memory: S_A [0,128), S_B [128,256), O_A [256, 256+D), O_B after.
+//   warp 9     tcgen05 issuer: ... S = Q_A K_j^T; O_A += P_A V_{j-1};
+//              S = Q_B K_j^T; O_B += P_B V_{j-1} ...  (S from shared memory
+//              operands, P from tensor memory).
+// Tensor memory: S [0,128) shared by the halves, P_A [128,192), P_B
+// [192,256) (16-bit pairs), O_A [256, 256+D), O_B after.  One S buffer
+// serves both halves because a half holds its S row in registers as soon as
+// the MMA has written it; with separate P buffers the next tile's Q K^T then
+// runs while the softmax of the current tile is still computing, so the
+// tensor pipe is not left waiting on the exponentials.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -49,12 +53,6 @@ namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 15.0f;  // log2 units: P stays <= 2^15 (fp16 range)
-// Optionally the two halves take turns for the exponential passes of a
-// tile, so that their softmax phases do not share the MUFU unit.  Measured
-// on B200 at 128K context it is 8% slower (the softmax of one half is longer
-// than the other half's MMAs), so it is off.
-constexpr bool kTakeTurns = false;
-
 // Share of the exponentials computed on the FMA pipe: pairs i with
 // (i % 8) < kPolyPerEight of each 16-pair chunk of a row.  Measured on B200
 // at 128K context: 0/8 14.3 ms, 2/8 14.6 ms, 3/8 15.2 ms (the polynomial's
@@ -83,7 +81,8 @@ struct Pf {
     static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;
     static constexpr int OFF_BAR = OFF_V + VST * TILE_BYTES;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;  // + barriers + align slack
-    static constexpr uint32_t S_COL = 0;          // S of half h at h * 128
+    static constexpr uint32_t S_COL = 0;          // S, shared by the halves
+    static constexpr uint32_t P_COL = 128;        // P of half h at 128 + h * 64
     static constexpr uint32_t O_COL = 256;        // O of half h at 256 + h * D
     static constexpr uint32_t TMEM_COLS = 512;
     static constexpr int THREADS = 320;
@@ -137,13 +136,14 @@ __device__ __forceinline__ int tile_key0(const Geom &G, int j)
 }
 
 struct Bars {
-    uint64_t q_full, q_empty, qloc_done;
+    uint64_t q_full, q_empty;
     uint64_t qh_full[2];
     uint64_t k_full[4], k_empty[4];
     uint64_t v_full[4], v_empty[4];
-    uint64_t s_full[2], p_full[2];
+    uint64_t s_full[2];  // S holds half h's scores of its current tile
+    uint64_t s_free[2];  // half h has read its S row into registers
+    uint64_t p_full[2];
     uint64_t o_bar[2], o_empty[2];
-    uint64_t turn[2];  // turn[h]: the other half finished its previous turn
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;  // set when any role gives up
@@ -199,31 +199,6 @@ __device__ __forceinline__ float2 exp2_poly2(float2 y)
                        __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
-// Key-validity mask of one 32-column chunk: x = -inf where key0 + e lies
-// outside [lo, hi].
-__device__ __forceinline__ void mask_chunk(float (&x)[32], int key0, int lo, int hi)
-{
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-        const int key = key0 + e;
-        if (key < lo || key > hi) x[e] = -INFINITY;
-    }
-}
-
-__device__ __forceinline__ float chunk_max(const float (&x)[32])
-{
-    float m[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) m[i] = fmax3(x[8 * i], x[8 * i + 1], x[8 * i + 2]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        m[i] = fmax3(m[i], x[8 * i + 3], x[8 * i + 4]);
-        m[i] = fmax3(m[i], x[8 * i + 5], x[8 * i + 6]);
-        m[i] = fmaxf(m[i], x[8 * i + 7]);
-    }
-    return fmaxf(fmaxf(m[0], m[1]), fmaxf(m[2], m[3]));
-}
-
 __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
 {
     uint32_t u[32];
@@ -233,8 +208,7 @@ __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
 }
 
 // Softmax numerators of one 32-column chunk: p = 2^(x c - m), packed to
-// 16-bit pairs (fp16 for core tiles, bf16 for raw ones) and stored to tensor
-// memory at p_addr (16 columns).  The MUFU unit computes 16 exponentials
+// 16-bit pairs in pk (fp16 for core tiles, bf16 for raw ones).  The MUFU unit computes 16 exponentials
 // per clock per SM, as many as the tile's MMAs need at full rate, so pairs
 // i with (i % 8) < kPolyPerEight take the FMA-pipe polynomial instead.  For
 // bf16 P (8 significant bits) the row sum adds exactly the rounded values
@@ -242,9 +216,8 @@ __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
 // O = (P V) / l; for fp16 P (11 bits) the fp32 values are summed.
 template <bool F16>
 __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float2 nm2,
-                                          uint32_t p_addr, float2 &acc)
+                                          uint32_t (&pk)[16], float2 &acc)
 {
-    uint32_t pk[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float2 y = __ffma2_rn(make_float2(x[2 * i], x[2 * i + 1]), c2, nm2);
@@ -259,7 +232,6 @@ __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float
             acc = __fadd2_rn(acc, make_float2(bf16_lo(pk[i]), bf16_hi(pk[i])));
         }
     }
-    tmem_st16(p_addr, pk);
 }
 
 __device__ __forceinline__ float row_max128(const float (&x)[128])
@@ -298,7 +270,6 @@ __global__ void __launch_bounds__(320, 1)
     if (threadIdx.x == 0) {
         mbar_init(&bars->q_full, 1);
         mbar_init(&bars->q_empty, 1);
-        mbar_init(&bars->qloc_done, 1);
         for (int s = 0; s < C::KST; ++s) {
             mbar_init(&bars->k_full[s], 1);
             mbar_init(&bars->k_empty[s], 1);
@@ -310,10 +281,10 @@ __global__ void __launch_bounds__(320, 1)
         for (int h = 0; h < 2; ++h) {
             mbar_init(&bars->qh_full[h], 4);
             mbar_init(&bars->s_full[h], 1);
+            mbar_init(&bars->s_free[h], 4);
             mbar_init(&bars->p_full[h], 4);
             mbar_init(&bars->o_bar[h], 1);
             mbar_init(&bars->o_empty[h], 4);
-            mbar_init(&bars->turn[h], 4);
         }
         mbar_init(&bars->mma_done, 1);
         bars->abort = 0;
@@ -415,7 +386,7 @@ __global__ void __launch_bounds__(320, 1)
             auto qk = [&](int hh, uint32_t s, bool core) {
                 const uint64_t a0 = dq + hh * kTile16, b0 = dk + s * kTile16;
                 const uint32_t idesc = core ? idesc_qk_h : idesc_qk_bf;
-                const uint32_t d_tmem = tmem + C::S_COL + hh * 128;
+                const uint32_t d_tmem = tmem + C::S_COL;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
                     constexpr uint32_t box16 = C::BOX_BYTES >> 4;
@@ -427,12 +398,14 @@ __global__ void __launch_bounds__(320, 1)
                 const uint64_t b0 = dv + sv * kTile16;
                 const uint32_t idesc = core ? idesc_pv_h : idesc_pv_bf;
                 const uint32_t d_tmem = tmem + C::O_COL + hh * D;
-                const uint32_t a_tmem = tmem + C::S_COL + hh * 128;
+                const uint32_t a_tmem = tmem + C::P_COL + hh * 64;
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk)
                     mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc,
                            (first && kk == 0) ? 0u : 1u);
             };
+            // it counts key tiles over all items; S is written once per half
+            // and tile, alternately A and B.
             for (int item = blockIdx.x; ok && item < p.n_items;
                  item += gridDim.x, ++k) {
                 const Geom G = geom(item, p);
@@ -457,25 +430,31 @@ __global__ void __launch_bounds__(320, 1)
                     }
                     return true;
                 };
-                for (int j = 0; ok && j < G.n_tiles; ++j) {
+                for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
                     const bool core = tile_is_core(G, j);
                     const uint32_t s = kc % C::KST;
                     if (!(ok = lane_wait(&bars->k_full[s], (kc / C::KST) & 1, bars))) break;
                     for (int hh = 0; hh < 2; ++hh) {
-                        if (j > 0 && !(ok = issue_pv(hh, j - 1))) break;
+                        // S is free once its previous occupant has been read:
+                        // half B's previous tile before S_A, half A's current
+                        // tile before S_B.
+                        if (hh == 1 || it > 0) {
+                            const uint32_t prev = hh == 0 ? it - 1 : it;
+                            if (!(ok = lane_wait(&bars->s_free[hh ^ 1], prev & 1, bars))) break;
+                        }
                         if (core && j == G.n_local &&
                             !(ok = lane_wait(&bars->qh_full[hh], cq & 1, bars)))
                             break;
                         tc_fence_after_sync();
                         qk(hh, s, core);
                         mma_commit(&bars->s_full[hh]);
+                        if (hh == 1) {
+                            mma_commit(&bars->k_empty[s]);
+                            ++kc;
+                            if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
+                        }
+                        if (j > 0 && !(ok = issue_pv(hh, j - 1))) break;
                     }
-                    if (!ok) break;
-                    mma_commit(&bars->k_empty[s]);
-                    ++kc;
-                    ++it;
-                    if (core_block && j == G.n_local - 1) mma_commit(&bars->qloc_done);
-                    if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
                 }
                 if (ok) ok = issue_pv(0, G.n_tiles - 1) && issue_pv(1, G.n_tiles - 1);
                 if (core_block) ++cq;
@@ -489,11 +468,11 @@ __global__ void __launch_bounds__(320, 1)
         const int hh = warp >> 2;                  // half
         const int row = threadIdx.x & 127;         // tensor-memory lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t s_addr = tmem + lane_off + C::S_COL + hh * 128;
+        const uint32_t s_addr = tmem + lane_off + C::S_COL;
+        const uint32_t p_addr = tmem + lane_off + C::P_COL + hh * 64;
         const uint32_t o_addr = tmem + lane_off + C::O_COL + hh * D;
-        uint32_t it = 0, pv_waits = 0, cq = 0;
+        uint32_t it = 0;  // key tiles over all items
         bool ok = true;
-        if (kTakeTurns && hh == 1 && lane == 0) mbar_arrive(&bars->turn[0]);  // A first
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
             const Geom G = geom(item, p);
             const bool core_block = G.n_core_tiles > 0;
@@ -513,95 +492,69 @@ __global__ void __launch_bounds__(320, 1)
                                             : (key0 < ws_hi || key0 + 127 > t0h);
                 const int lo = core ? 0 : ws_t;
                 const int hi = core ? nc_t - 1 : t;
-                if (kTakeTurns && !(ok = warp_wait(&bars->turn[hh], it & 1, bars))) break;
-                // pass 1: row maximum of the tile (one 128-column load)
-                float mx;
+                // The whole S row into registers; S is then free for the
+                // other half's next Q K^T.
+                float x[128];
                 {
-                    float x[128];
-                    {
-                        uint32_t u[128];
-                        tmem_ld128_wait(s_addr, u);
+                    uint32_t u[128];
+                    tmem_ld128_wait(s_addr, u);
 #pragma unroll
-                        for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
-                    }
-                    if (need_mask) {
-#pragma unroll
-                        for (int e = 0; e < 128; ++e) {
-                            const int key = key0 + e;
-                            if (key < lo || key > hi) x[e] = -INFINITY;
-                        }
-                    }
-                    mx = row_max128(x);
+                    for (int e = 0; e < 128; ++e) x[e] = __uint_as_float(u[e]);
                 }
-                const float m_tile = mx * p.scale_log2;
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s_free[hh]);
+                if (need_mask) {
+#pragma unroll
+                    for (int e = 0; e < 128; ++e) {
+                        const int key = key0 + e;
+                        if (key < lo || key > hi) x[e] = -INFINITY;
+                    }
+                }
+                const float m_tile = row_max128(x) * p.scale_log2;
                 float alpha = 1.f;
                 if (m_tile > m_run + kRescaleThreshold) {
                     alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_tile);
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                // pass 2: P = 2^(S c - m) over the S columns already read
-                // (chunk c's 32 logits become 16 packed columns at c*16, below
-                // the chunks still to be read; the MMA reads P only after
-                // p_full below).
+                // P V of the previous tile (over all items) must have read
+                // P_h and written O_h before either is touched.  Waiting here
+                // lets each chunk of P go to tensor memory as soon as it is
+                // computed; holding all of P in registers until after the
+                // exponentials spills registers and measured 4% slower on
+                // B200 at 128K context.
+                if (it > 0) {
+                    if (!(ok = warp_wait(&bars->o_bar[hh], (it - 1) & 1, bars))) break;
+                    tc_fence_after_sync();
+                }
+                // P = 2^(S c - m), packed and written chunk by chunk
                 const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 acc = make_float2(0.f, 0.f);
-                // Chunks are read in pairs, the second chunk's load in flight
-                // while the first is processed (a wait covers every earlier
-                // load, so the second load is issued after the first wait).
-                // The loop over the pairs stays rolled: fully unrolled, the
-                // softmax code outgrows the instruction cache.
-#pragma unroll 1
-                for (int c = 0; c < 4; c += 2) {
-                    uint32_t ua[32], ub[32];
-                    tmem_ld32(s_addr + c * 32, ua);
-                    tmem_wait_ld_dep(ua);
-                    tmem_ld32(s_addr + (c + 1) * 32, ub);
-                    {
-                        float x[32];
+                uint32_t pk[4][16];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ua[e]);
-                        if (need_mask) mask_chunk(x, key0 + c * 32, lo, hi);
-                        if (core)
-                            exp_chunk<true>(x, c2, nm2, s_addr + c * 16, acc);
-                        else
-                            exp_chunk<false>(x, c2, nm2, s_addr + c * 16, acc);
-                    }
-                    tmem_wait_ld_dep(ub);
-                    {
-                        float x[32];
+                for (int c = 0; c < 4; ++c) {
+                    float xc[32];
 #pragma unroll
-                        for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(ub[e]);
-                        if (need_mask) mask_chunk(x, key0 + (c + 1) * 32, lo, hi);
-                        if (core)
-                            exp_chunk<true>(x, c2, nm2, s_addr + (c + 1) * 16, acc);
-                        else
-                            exp_chunk<false>(x, c2, nm2, s_addr + (c + 1) * 16, acc);
-                    }
+                    for (int e = 0; e < 32; ++e) xc[e] = x[c * 32 + e];
+                    if (core)
+                        exp_chunk<true>(xc, c2, nm2, pk[c], acc);
+                    else
+                        exp_chunk<false>(xc, c2, nm2, pk[c], acc);
+                    tmem_st16(p_addr + c * 16, pk[c]);
                 }
-                const float rs = acc.x + acc.y;
-                if (kTakeTurns) {
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&bars->turn[hh ^ 1]);
-                }
-                l_run = fmaf(l_run, alpha, rs);
-                if (j > 0) {
-                    // P V of the previous tile is complete (it was issued
-                    // before this tile's S); rescale O if the max moved
-                    if (!(ok = warp_wait(&bars->o_bar[hh], pv_waits & 1, bars))) break;
-                    ++pv_waits;
-                    tc_fence_after_sync();
-                    if (__any_sync(0xffffffffu, alpha != 1.f)) {
+                l_run = fmaf(l_run, alpha, acc.x + acc.y);
+                // the max moved (rare): rescale O before P V of this tile
+                if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-                        for (int c = 0; c < D / 32; ++c) {
-                            uint32_t u[32];
-                            tmem_ld32_wait(o_addr + c * 32, u);
+                    for (int c = 0; c < D / 32; ++c) {
+                        uint32_t u[32];
+                        tmem_ld32_wait(o_addr + c * 32, u);
 #pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
-                            tmem_st32(o_addr + c * 32, u);
-                        }
+                        for (int e = 0; e < 32; ++e)
+                            u[e] = __float_as_uint(__uint_as_float(u[e]) * alpha);
+                        tmem_st32(o_addr + c * 32, u);
                     }
                 }
                 tmem_wait_st();
@@ -609,11 +562,11 @@ __global__ void __launch_bounds__(320, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&bars->p_full[hh]);
                 if (core_block && j == G.n_local - 1) {
-                    // Last local tile done: once every local Q K^T has read
-                    // the bf16 Q block, turn this half into fp16 in place for
-                    // the core stream (16-byte chunks of 8 elements keep
-                    // their swizzled places).
-                    if (!(ok = warp_wait(&bars->qloc_done, cq & 1, bars))) break;
+                    // Last local tile: its Q K^T, the last reader of the bf16
+                    // Q half, is complete (its S was ready), so turn this
+                    // half into fp16 in place for the core stream (16-byte
+                    // chunks of 8 elements keep their swizzled places).  The
+                    // first core Q K^T of the half waits for this.
                     bool over = false;
                     uint4 *q4 = reinterpret_cast<uint4 *>(sQ + hh * C::TILE_BYTES);
 #pragma unroll 4
@@ -633,10 +586,9 @@ __global__ void __launch_bounds__(320, 1)
                 }
             }
             if (!ok) break;
-            if (core_block) ++cq;
-            // Epilogue: O / l for this row.
-            if (!(ok = warp_wait(&bars->o_bar[hh], pv_waits & 1, bars))) break;
-            ++pv_waits;
+            // Epilogue: O / l for this row, once P V of the item's last
+            // tile (tile it - 1) is complete.
+            if (!(ok = warp_wait(&bars->o_bar[hh], (it - 1) & 1, bars))) break;
             tc_fence_after_sync();
             // O / l for this row, 32 columns at a time; O is read completely
             // before its tensor memory is released
