@@ -55,8 +55,9 @@ constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 15.0f;  // log2 units: P stays <= 2^15 (fp16 range)
 // Share of the exponentials computed on the FMA pipe: pairs i with
 // (i % 8) < kPolyPerEight of each 16-pair chunk of a row.  Measured on B200
-// at 128K context: 0/8 14.3 ms, 2/8 14.6 ms, 3/8 15.2 ms (the polynomial's
-// extra issue slots cost more than the MUFU time it frees), so it is 0.
+// at 128K context against 0/8: 2/8 +7%, 3/8 +8%, 4/8 +11% time (the
+// exponentials run beside the MMAs, so freeing MUFU time gains nothing and
+// the polynomial's extra instructions cost), so it is 0.
 constexpr int kPolyPerEight = 0;
 
 // 2^f on [-1/2, 1/2] by a degree-3 polynomial whose coefficients were fitted

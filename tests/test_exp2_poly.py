@@ -1,6 +1,7 @@
 """The FMA-pipe exp2 of the prefill kernel, replayed in float32 on the CPU.
 
-The kernel computes part of its softmax exponentials as 2^y = 2^n * p(f)
+The kernel can compute a share of its softmax exponentials (kPolyPerEight
+of every eight pairs; currently none) as 2^y = 2^n * p(f)
 with n = rint(y) taken from the low mantissa bits of y + 1.5*2^23,
 f = y - n in [-1/2, 1/2], p a degree-3 polynomial, and n added to the
 exponent field of p(f).  This test reads the polynomial's coefficients and
