@@ -453,7 +453,7 @@ def main(argv=None) -> int:
                             for t in range(DECODE.T, DECODE.T + DECODE.steps)]))
     dec_gbs = dbytes / (nz(dec_us) * 1e-6) / 1e9
     pool_gbs = pbytes / (nz(r["pool_ms"]) * 1e-3) / 1e9
-    launches = args.steps * ((2 if do_prefill else 0) + (3 * DECODE.steps if do_decode else 0))
+    launches = args.steps * ((2 if do_prefill else 0) + (2 * DECODE.steps if do_decode else 0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
@@ -481,7 +481,7 @@ def main(argv=None) -> int:
                          "frac": pool_gbs / pk["hbm_gbs"], "bytes": pbytes},
             "decode_step": {"us": dec_us, "gbs": dec_gbs, "frac": dec_gbs / pk["hbm_gbs"],
                             "bytes": dbytes,
-                            "launches": "cca_cache_append + cca_attn_decode (split + merge)"},
+                            "launches": "cca_cache_append + cca_attn_decode (ticket memset + split kernel with fused merge)"},
         },
         "kv_cache": cache_bytes(pw, pw.T),
         "clocks": r["clocks"],

@@ -156,7 +156,9 @@ size_t cca_decode_workspace_bytes(const cca_cache *c);
  *   q_t [B, Hq, d] (bf16), o_t [B, Hq, d] written in o_dtype.
  * Split over key ranges; partial results go to `workspace` (device memory
  * of at least cca_decode_workspace_bytes(c) bytes, 256-byte aligned, its
- * contents need no initialisation), then a merge kernel combines them.
+ * contents need no initialisation: the call clears the few counters it
+ * uses with cudaMemsetAsync on `stream`).  The last block of each (batch,
+ * kv head) to finish combines the partials, in the same kernel.
  */
 cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                            cca_dtype o_dtype, void *workspace,

@@ -159,7 +159,7 @@ cca_status cca_cache_append(cca_cache *c, const void *q_t, const void *k_t,
 size_t cca_decode_workspace_bytes(const cca_cache *c)
 {
     if (cache_status(c) != CCA_OK) return 0;
-    return cca::decode_workspace_bytes(c->B, c->Hq, c->d, c->core_cap, c->tail_cap);
+    return cca::decode_workspace_bytes(c->B, c->Hq, c->Hkv, c->d, c->core_cap, c->tail_cap);
 }
 
 cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
@@ -173,7 +173,7 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
     if (!ptr_ok(q_t, true) || !ptr_ok(o_t, true) || workspace == nullptr ||
         (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
         return CCA_ERR_INVALID_ARG;
-    if (workspace_bytes < cca::decode_workspace_bytes(c->B, c->Hq, c->d, c->core_cap,
+    if (workspace_bytes < cca::decode_workspace_bytes(c->B, c->Hq, c->Hkv, c->d, c->core_cap,
                                                       c->tail_cap))
         return CCA_ERR_INVALID_ARG;
     const int64_t t = c->len - 1;

@@ -8,7 +8,9 @@
 // HBM-bound split-K GEMV: the keys of one (batch, key/value head) are cut
 // into chunks; one CTA streams one chunk's K and V rows once for all r query
 // heads of that key/value head, producing a partial (max, sum, unnormalised
-// output) per query head; a merge kernel rescales and adds the partials.
+// output) per query head.  The last CTA of a (batch, key/value head) to
+// finish, found by an atomic ticket, rescales and adds the partials and
+// writes the output: one launch, no separate merge kernel.
 #include "common.cuh"
 #include "internal.h"
 
@@ -68,8 +70,9 @@ template <int D, int R>
 __global__ void __launch_bounds__(kDecodeThreads)
     decode_split_kernel(CacheView cv, const uint16_t *__restrict__ q_t,
                         float *__restrict__ part_o, float2 *__restrict__ part_ml,
-                        int Hq, int Hkv, int64_t n_keys, int chunk, int nsplit,
-                        float scale_log2)
+                        unsigned int *__restrict__ tickets, void *__restrict__ o_t,
+                        int out_f32, int Hq, int Hkv, int64_t n_keys, int chunk,
+                        int nsplit, float scale_log2)
 {
     using S = DecodeShape<D>;
     extern __shared__ float dsm[];
@@ -207,76 +210,92 @@ __global__ void __launch_bounds__(kDecodeThreads)
         part_o[qrow * D + c] = s;
         if (c == 0) part_ml[qrow] = make_float2(stat[2 * k], stat[2 * k + 1]);
     }
-}
 
-// One warp per (batch, query head): combine the splits' partials.  Lanes
-// take the splits in parallel for the maximum and the weights
-// 2^(m_s - max), which go to shared memory; then each lane adds its D/32
-// output dims over the splits with independent loads.
-constexpr int kMergeWarps = 4;
+    // Ticket: the CTA that takes the last one merges.  The fence makes this
+    // CTA's partials visible device-wide before its ticket is counted.
+    __threadfence();
+    __syncthreads();
+    __shared__ unsigned int last;
+    if (tid == 0) last = atomicAdd(&tickets[bh], 1u) == static_cast<unsigned int>(nsplit - 1);
+    __syncthreads();
+    if (!last) return;
+    __threadfence();
 
-template <int D>
-__global__ void __launch_bounds__(kMergeWarps * 32)
-    decode_merge_kernel(const float *__restrict__ part_o,
-                        const float2 *__restrict__ part_ml, void *__restrict__ o_t,
-                        int out_f32, int64_t rows, int nsplit)
-{
-    constexpr int DPL = D / 32;
-    extern __shared__ float merge_w[];  // [kMergeWarps][nsplit]
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t row = static_cast<int64_t>(blockIdx.x) * kMergeWarps + warp;
-    if (row >= rows) return;
-    float *w = merge_w + warp * nsplit;
-    const float2 *ml = part_ml + row * nsplit;
-    float mx = -INFINITY;
-    for (int s = lane; s < nsplit; s += 32) mx = fmaxf(mx, ml[s].x);
-    mx = warp_max(mx);
-    float l = 0.f;
-    for (int s = lane; s < nsplit; s += 32) {
-        const float2 v = ml[s];
-        const float c = fast_exp2(v.x - mx);
-        w[s] = c;
-        l = fmaf(c, v.y, l);
-    }
-    l = warp_sum(l);
-    __syncwarp();
-    float acc[DPL];
-#pragma unroll
-    for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
-    const float *po = part_o + row * nsplit * D + lane * DPL;
-#pragma unroll 4
-    for (int s = 0; s < nsplit; ++s) {
-        const float c = w[s];
-        const float *src = po + static_cast<int64_t>(s) * D;
-        if constexpr (DPL == 4) {
-            const float4 v = *reinterpret_cast<const float4 *>(src);
-            acc[0] = fmaf(c, v.x, acc[0]);
-            acc[1] = fmaf(c, v.y, acc[1]);
-            acc[2] = fmaf(c, v.z, acc[2]);
-            acc[3] = fmaf(c, v.w, acc[3]);
-        } else {
-            const float2 v = *reinterpret_cast<const float2 *>(src);
-            acc[0] = fmaf(c, v.x, acc[0]);
-            acc[1] = fmaf(c, v.y, acc[1]);
+    // Merge, per query head k: M = max_s m_s, L = sum_s 2^(m_s - M) l_s,
+    // o = sum_s 2^(m_s - M) o_s / L.  Partials are read from L2 (__ldcg):
+    // other CTAs wrote them.  The weights 2^(m_s - M) go to shared memory
+    // (the score buffer, free now) when they fit; every thread then keeps
+    // several independent 16-byte loads of partial outputs in flight.
+    const bool wfit = nsplit <= chunk;
+    for (int k = warp; k < r; k += kDecodeThreads / 32) {
+        const float2 *ml = part_ml + (b * Hq + h * r + k) * nsplit;
+        float mx = -INFINITY;
+        for (int sp = lane; sp < nsplit; sp += 32) mx = fmaxf(mx, __ldcg(&ml[sp].x));
+        mx = warp_max(mx);
+        float l = 0.f;
+        for (int sp = lane; sp < nsplit; sp += 32) {
+            const float2 v = __ldcg(&ml[sp]);
+            const float wgt = fast_exp2(v.x - mx);
+            if (wfit) lg[k * chunk + sp] = wgt;
+            l = fmaf(wgt, v.y, l);
+        }
+        l = warp_sum(l);
+        if (lane == 0) {
+            stat[2 * k] = mx;
+            stat[2 * k + 1] = 1.0f / l;
         }
     }
-    const float inv = 1.0f / l;
-    if (out_f32) {
-        float *o = static_cast<float *>(o_t) + row * D + lane * DPL;
+    __syncthreads();
+    constexpr int C4 = D / 4;                    // float4 columns of a row
+    constexpr int SG = kDecodeThreads / C4;      // splits taken at once
+    float4 *red4 = reinterpret_cast<float4 *>(red);  // [SG][C4]
+    const int c4 = tid % C4, g0 = tid / C4;
+    for (int k = 0; k < r; ++k) {
+        const int64_t orow = b * Hq + h * r + k;
+        const float2 *ml = part_ml + orow * nsplit;
+        const float4 *po4 = reinterpret_cast<const float4 *>(part_o + orow * nsplit * D) + c4;
+        const float mx = stat[2 * k];
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+        for (int sp = g0; sp < nsplit; sp += SG) {
+            const float wgt = wfit ? lg[k * chunk + sp] : fast_exp2(__ldcg(&ml[sp].x) - mx);
+            const float4 v = __ldcg(po4 + static_cast<int64_t>(sp) * C4);
+            acc.x = fmaf(wgt, v.x, acc.x);
+            acc.y = fmaf(wgt, v.y, acc.y);
+            acc.z = fmaf(wgt, v.z, acc.z);
+            acc.w = fmaf(wgt, v.w, acc.w);
+        }
+        red4[g0 * C4 + c4] = acc;
+        __syncthreads();
+        if (tid < C4) {
+            float4 o = red4[tid];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) o[e] = acc[e] * inv;
-    } else {
-        uint16_t *o = static_cast<uint16_t *>(o_t) + row * D + lane * DPL;
-#pragma unroll
-        for (int e = 0; e < DPL; e += 2)
-            *reinterpret_cast<uint32_t *>(o + e) = pack_bf16x2(acc[e] * inv, acc[e + 1] * inv);
+            for (int gi = 1; gi < SG; ++gi) {
+                const float4 v = red4[gi * C4 + tid];
+                o.x += v.x;
+                o.y += v.y;
+                o.z += v.z;
+                o.w += v.w;
+            }
+            const float inv = stat[2 * k + 1];
+            if (out_f32) {
+                reinterpret_cast<float4 *>(static_cast<float *>(o_t) + orow * D)[tid] =
+                    make_float4(o.x * inv, o.y * inv, o.z * inv, o.w * inv);
+            } else {
+                reinterpret_cast<uint2 *>(static_cast<uint16_t *>(o_t) + orow * D)[tid] =
+                    make_uint2(pack_bf16x2(o.x * inv, o.y * inv),
+                               pack_bf16x2(o.z * inv, o.w * inv));
+            }
+        }
+        __syncthreads();
     }
 }
 
 template <int D, int R>
 cudaError_t launch_split(const CacheView &cv, const void *q_t, float *part_o,
-                         float2 *part_ml, int B, int Hq, int Hkv, int64_t n_keys,
-                         int nsplit, float scale_log2, cudaStream_t s)
+                         float2 *part_ml, unsigned int *tickets, void *o_t, bool o_f32,
+                         int B, int Hq, int Hkv, int64_t n_keys, int nsplit,
+                         float scale_log2, cudaStream_t s)
 {
     using S = DecodeShape<D>;
     const size_t smem =
@@ -287,8 +306,9 @@ cudaError_t launch_split(const CacheView &cv, const void *q_t, float *part_o,
                              static_cast<int>(smem));
     dim3 grid(nsplit, B * Hkv);
     kern<<<grid, kDecodeThreads, smem, s>>>(cv, static_cast<const uint16_t *>(q_t),
-                                            part_o, part_ml, Hq, Hkv, n_keys,
-                                            kDecodeChunk, nsplit, scale_log2);
+                                            part_o, part_ml, tickets, o_t, o_f32 ? 1 : 0,
+                                            Hq, Hkv, n_keys, kDecodeChunk, nsplit,
+                                            scale_log2);
     return cudaGetLastError();
 }
 
@@ -312,14 +332,28 @@ int decode_max_splits(int64_t core_cap, int64_t tail_cap)
     return static_cast<int>((core_cap + tail_cap + kDecodeChunk - 1) / kDecodeChunk);
 }
 
-size_t decode_workspace_bytes(int B, int Hq, int d, int64_t core_cap,
-                              int64_t tail_cap)
+// Workspace: part_o [B, Hq, splits, d] fp32 | part_ml [B, Hq, splits] (max,
+// sum) | tickets [B * Hkv] u32, each part 256-byte aligned.
+namespace {
+struct WorkspaceLayout {
+    size_t o_bytes, ml_bytes, ticket_bytes;
+};
+WorkspaceLayout workspace_layout(int B, int Hq, int Hkv, int d, int64_t core_cap,
+                                 int64_t tail_cap)
 {
     const size_t rows = static_cast<size_t>(B) * Hq *
                         static_cast<size_t>(decode_max_splits(core_cap, tail_cap));
-    size_t o_bytes = rows * d * sizeof(float);
-    o_bytes = (o_bytes + 255) / 256 * 256;
-    return o_bytes + rows * sizeof(float2);
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return {up(rows * d * sizeof(float)), up(rows * sizeof(float2)),
+            up(static_cast<size_t>(B) * Hkv * sizeof(unsigned int))};
+}
+}  // namespace
+
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t core_cap,
+                              int64_t tail_cap)
+{
+    const WorkspaceLayout L = workspace_layout(B, Hq, Hkv, d, core_cap, tail_cap);
+    return L.o_bytes + L.ml_bytes + L.ticket_bytes;
 }
 
 cudaError_t launch_decode(const void *k_core, const void *v_core,
@@ -330,12 +364,11 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
                           int64_t t, cudaStream_t s)
 {
     const DecodePlan p = decode_plan(t, g, w, B, Hkv);
-    const int maxs = decode_max_splits(core_cap, tail_cap);
-    const size_t rows_max = static_cast<size_t>(B) * Hq * maxs;
-    size_t o_bytes = rows_max * d * sizeof(float);
-    o_bytes = (o_bytes + 255) / 256 * 256;
-    float *part_o = static_cast<float *>(workspace);
-    float2 *part_ml = reinterpret_cast<float2 *>(static_cast<char *>(workspace) + o_bytes);
+    const WorkspaceLayout L = workspace_layout(B, Hq, Hkv, d, core_cap, tail_cap);
+    char *ws = static_cast<char *>(workspace);
+    float *part_o = reinterpret_cast<float *>(ws);
+    float2 *part_ml = reinterpret_cast<float2 *>(ws + L.o_bytes);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + L.o_bytes + L.ml_bytes);
     CacheView cv{static_cast<const uint16_t *>(k_core),
                  static_cast<const uint16_t *>(v_core),
                  static_cast<const uint16_t *>(k_tail),
@@ -346,10 +379,13 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
                  p.n_core};
     const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
     const int r = Hq / Hkv;
-    cudaError_t e;
+    // the tickets start at zero on every call (the workspace is not
+    // assumed to hold anything)
+    cudaError_t e = cudaMemsetAsync(tickets, 0, sizeof(unsigned int) * B * Hkv, s);
+    if (e != cudaSuccess) return e;
 #define CCA_SPLIT(DD, RR)                                                          \
-    e = launch_split<DD, RR>(cv, q_t, part_o, part_ml, B, Hq, Hkv, p.n_keys,     \
-                             p.nsplit, scale_log2, s)
+    e = launch_split<DD, RR>(cv, q_t, part_o, part_ml, tickets, o_t, o_f32, B, Hq, \
+                             Hkv, p.n_keys, p.nsplit, scale_log2, s)
     if (d == 128) {
         if (r == 1) CCA_SPLIT(128, 1);
         else if (r == 2) CCA_SPLIT(128, 2);
@@ -364,17 +400,7 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
         else CCA_SPLIT(64, 16);
     }
 #undef CCA_SPLIT
-    if (e != cudaSuccess) return e;
-    const int64_t rows = static_cast<int64_t>(B) * Hq;
-    const int blocks = static_cast<int>((rows + kMergeWarps - 1) / kMergeWarps);
-    const size_t msmem = sizeof(float) * kMergeWarps * p.nsplit;
-    if (d == 128)
-        decode_merge_kernel<128><<<blocks, kMergeWarps * 32, msmem, s>>>(
-            part_o, part_ml, o_t, o_f32 ? 1 : 0, rows, p.nsplit);
-    else
-        decode_merge_kernel<64><<<blocks, kMergeWarps * 32, msmem, s>>>(
-            part_o, part_ml, o_t, o_f32 ? 1 : 0, rows, p.nsplit);
-    return cudaGetLastError();
+    return e;
 }
 
 }  // namespace cca

@@ -15,9 +15,10 @@
 // current, on that device's first call (cudaGetSymbolAddress).  That first
 // call should therefore come before any stream capture begins.  The contents
 // left by one call are simply overwritten by the next: every partial result
-// the merge reads is written earlier in the same call, so nothing needs to
-// start at zero.  All calls share the one array, so calls whose kernels
-// overlap on the GPU (different streams, no ordering between them) race.
+// the merge reads is written earlier in the same call, and the call clears
+// its own completion counters, so nothing needs to start at zero.  All calls
+// share the one array, so calls whose kernels overlap on the GPU (different
+// streams, no ordering between them) race.
 #include <mutex>
 
 #include "../../include/cca.h"

@@ -39,7 +39,7 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(int64_t t, int g, int w, int B, int Hkv);
 int decode_max_splits(int64_t core_cap, int64_t tail_cap);
-size_t decode_workspace_bytes(int B, int Hq, int d, int64_t core_cap,
+size_t decode_workspace_bytes(int B, int Hq, int Hkv, int d, int64_t core_cap,
                               int64_t tail_cap);
 cudaError_t launch_decode(const void *k_core, const void *v_core,
                           const void *k_tail, const void *v_tail,
