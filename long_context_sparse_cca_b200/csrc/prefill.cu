@@ -17,8 +17,8 @@
 // Blocks are dealt round-robin to one persistent CTA per SM, latest blocks
 // (most core tiles) first.
 //
-// CTA of 320 threads (168 registers a thread: registers are booked for warps
-// in groups of four, so ten warps count as twelve):
+// CTA of 352 threads (168 registers a thread: registers are booked for warps
+// in groups of four, so eleven warps count as twelve):
 //   warps 0-3  softmax of half A, warps 4-7 softmax of half B: thread i owns
 //              query row i of its half; copies its S row from tensor memory
 //              into registers (which frees S for the next Q K^T), masks,
@@ -29,9 +29,13 @@
 //              half of the Q tile from bf16 into fp16 in place.
 //   warp 8     TMA producer: the Q block, then per key tile one K and one V
 //              tile into multi-stage shared-memory rings (128-byte swizzle).
-//   warp 9     tcgen05 issuer: ... S = Q_A K_j^T; O_A += P_A V_{j-1};
-//              S = Q_B K_j^T; O_B += P_B V_{j-1} ...  (S from shared memory
-//              operands, P from tensor memory).
+//   warp 9     Q K^T issuer: ... S = Q_A K_j^T; S = Q_B K_j^T ...  (both
+//              operands from shared memory).
+//   warp 10    P V issuer: ... O_A += P_A V_j; O_B += P_B V_j ...  (P from
+//              tensor memory).  An MMA-issuing thread stalls the tensor pipe
+//              whenever it waits on a barrier, even one already complete;
+//              with two issuers one keeps the pipe busy while the other
+//              waits.
 // Tensor memory: S [0,128) shared by the halves, P_A [128,192), P_B
 // [192,256) (16-bit pairs), O_A [256, 256+D), O_B after.  One S buffer
 // serves both halves because a half holds its S row in registers as soon as
@@ -86,7 +90,7 @@ struct Pf {
     static constexpr uint32_t P_COL = 128;        // P of half h at 128 + h * 64
     static constexpr uint32_t O_COL = 256;        // O of half h at 256 + h * D
     static constexpr uint32_t TMEM_COLS = 512;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 352;
 };
 
 struct Params {
@@ -145,7 +149,7 @@ struct Bars {
     uint64_t s_free[2];  // half h has read its S row into registers
     uint64_t p_full[2];
     uint64_t o_bar[2], o_empty[2];
-    uint64_t mma_done;
+    uint64_t mma_done, mma_done2;  // Q K^T issuer, P V issuer
     uint32_t tmem_base;
     int abort;  // set when any role gives up
     int never;  // stays 0: drain waits are bounded by time only
@@ -250,7 +254,7 @@ __device__ __forceinline__ float row_max128(const float (&x)[128])
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(352, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV,
@@ -288,6 +292,7 @@ __global__ void __launch_bounds__(320, 1)
             mbar_init(&bars->o_empty[h], 4);
         }
         mbar_init(&bars->mma_done, 1);
+        mbar_init(&bars->mma_done2, 1);
         bars->abort = 0;
         bars->never = 0;
         mbar_fence_init();
@@ -366,103 +371,112 @@ __global__ void __launch_bounds__(320, 1)
             }
             if (qc > 0) wait_bounded(&bars->q_full, (qc - 1) & 1, never, kWaitLimitNs);
         }
-    } else if (warp == 9) {
-        // ------------------------------------------------ tcgen05 issuer
+    } else if (warp == 9 || warp == 10) {
+        // ------------------------------------------------ tcgen05 issuers
+        // Warp 9 issues S = Q K^T, warp 10 issues O += P V.  A thread that
+        // issues MMAs stalls the tensor pipe while it waits on a barrier
+        // (even a completed one); with two issuers one keeps the pipe busy
+        // while the other waits.
         if (lane == 0) {
             constexpr uint32_t idesc_qk_bf = idesc_f32acc(128, 128, true, false, false);
             constexpr uint32_t idesc_qk_h = idesc_f32acc(128, 128, false, false, false);
             constexpr uint32_t idesc_pv_bf = idesc_f32acc(128, D, true, false, true);
             constexpr uint32_t idesc_pv_h = idesc_f32acc(128, D, false, false, true);
-            const uint32_t q_base = smem_addr(sQ), k_base = smem_addr(sK),
-                           v_base = smem_addr(sV);
-            uint32_t kc = 0, vc = 0, it = 0, cq = 0;
-            int k = 0;
-            bool ok = true;
             // Shared-memory descriptors: the start-address field (bits
             // 0-13, 16-byte units) is advanced by plain addition.
-            const uint64_t dq = smem_desc_sw128(q_base, 16, 1024);
-            const uint64_t dk = smem_desc_sw128(k_base, 16, 1024);
-            const uint64_t dv = smem_desc_sw128(v_base, C::BOX_BYTES, 1024);
+            const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(sV), C::BOX_BYTES, 1024);
             constexpr uint32_t kTile16 = C::TILE_BYTES >> 4;
-            auto qk = [&](int hh, uint32_t s, bool core) {
-                const uint64_t a0 = dq + hh * kTile16, b0 = dk + s * kTile16;
-                const uint32_t idesc = core ? idesc_qk_h : idesc_qk_bf;
-                const uint32_t d_tmem = tmem + C::S_COL;
+            uint32_t it = 0;  // key tiles over all items
+            int k = 0;
+            bool ok = true;
+            if (warp == 9) {
+                uint32_t kc = 0, cq = 0;
+                auto qk = [&](int hh, uint32_t s, bool core) {
+                    const uint64_t a0 = dq + hh * kTile16, b0 = dk + s * kTile16;
+                    const uint32_t idesc = core ? idesc_qk_h : idesc_qk_bf;
+                    const uint32_t d_tmem = tmem + C::S_COL;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    constexpr uint32_t box16 = C::BOX_BYTES >> 4;
-                    const uint32_t off = (kk >> 2) * box16 + (kk & 3) * 2;
-                    mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        constexpr uint32_t box16 = C::BOX_BYTES >> 4;
+                        const uint32_t off = (kk >> 2) * box16 + (kk & 3) * 2;
+                        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+                    }
+                };
+                for (int item = blockIdx.x; ok && item < p.n_items;
+                     item += gridDim.x, ++k) {
+                    const Geom G = geom(item, p);
+                    if (!(ok = lane_wait(&bars->q_full, k & 1, bars))) break;
+                    for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
+                        const bool core = tile_is_core(G, j);
+                        const uint32_t s = kc % C::KST;
+                        if (!(ok = lane_wait(&bars->k_full[s], (kc / C::KST) & 1, bars))) break;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            // S is free once its previous occupant has been
+                            // read: half B's previous tile before S_A, half
+                            // A's current tile before S_B.
+                            if (hh == 1 || it > 0) {
+                                const uint32_t prev = hh == 0 ? it - 1 : it;
+                                if (!(ok = lane_wait(&bars->s_free[hh ^ 1], prev & 1, bars)))
+                                    break;
+                            }
+                            if (core && j == G.n_local &&
+                                !(ok = lane_wait(&bars->qh_full[hh], cq & 1, bars)))
+                                break;
+                            tc_fence_after_sync();
+                            qk(hh, s, core);
+                            mma_commit(&bars->s_full[hh]);
+                        }
+                        if (!ok) break;
+                        mma_commit(&bars->k_empty[s]);
+                        ++kc;
+                        if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
+                    }
+                    if (G.n_core_tiles > 0) ++cq;
                 }
-            };
-            auto pv = [&](int hh, uint32_t sv, bool core, bool first) {
-                const uint64_t b0 = dv + sv * kTile16;
-                const uint32_t idesc = core ? idesc_pv_h : idesc_pv_bf;
-                const uint32_t d_tmem = tmem + C::O_COL + hh * D;
-                const uint32_t a_tmem = tmem + C::P_COL + hh * 64;
+                // Wait for every Q K^T this thread issued to finish.
+                mma_commit(&bars->mma_done);
+                wait_bounded(&bars->mma_done, 0, &bars->never, kWaitLimitNs);
+            } else {
+                uint32_t vc = 0;
+                auto pv = [&](int hh, uint32_t sv, bool core, bool first) {
+                    const uint64_t b0 = dv + sv * kTile16;
+                    const uint32_t idesc = core ? idesc_pv_h : idesc_pv_bf;
+                    const uint32_t d_tmem = tmem + C::O_COL + hh * D;
+                    const uint32_t a_tmem = tmem + C::P_COL + hh * 64;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc,
-                           (first && kk == 0) ? 0u : 1u);
-            };
-            // it counts key tiles over all items; S is written once per half
-            // and tile, alternately A and B.
-            for (int item = blockIdx.x; ok && item < p.n_items;
-                 item += gridDim.x, ++k) {
-                const Geom G = geom(item, p);
-                const bool core_block = G.n_core_tiles > 0;
-                if (!(ok = lane_wait(&bars->q_full, k & 1, bars))) break;
-                const uint32_t it0 = it;
-                // P V of tile jj for half hh (V stage waited by half A).
-                auto issue_pv = [&](int hh, int jj) -> bool {
-                    const uint32_t itp = it0 + jj;
-                    if (!lane_wait(&bars->p_full[hh], itp & 1, bars)) return false;
-                    if (jj == 0 && k > 0 && !lane_wait(&bars->o_empty[hh], (k - 1) & 1, bars))
-                        return false;
-                    const uint32_t sv = vc % C::VST;
-                    if (hh == 0 && !lane_wait(&bars->v_full[sv], (vc / C::VST) & 1, bars))
-                        return false;
-                    tc_fence_after_sync();
-                    pv(hh, sv, tile_is_core(G, jj), jj == 0);
-                    mma_commit(&bars->o_bar[hh]);
-                    if (hh == 1) {
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc,
+                               (first && kk == 0) ? 0u : 1u);
+                };
+                for (int item = blockIdx.x; ok && item < p.n_items;
+                     item += gridDim.x, ++k) {
+                    const Geom G = geom(item, p);
+                    for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
+                        const bool core = tile_is_core(G, j);
+                        const uint32_t sv = vc % C::VST;
+                        for (int hh = 0; hh < 2; ++hh) {
+                            if (!(ok = lane_wait(&bars->p_full[hh], it & 1, bars))) break;
+                            if (j == 0 && k > 0 &&
+                                !(ok = lane_wait(&bars->o_empty[hh], (k - 1) & 1, bars)))
+                                break;
+                            if (hh == 0 &&
+                                !(ok = lane_wait(&bars->v_full[sv], (vc / C::VST) & 1, bars)))
+                                break;
+                            tc_fence_after_sync();
+                            pv(hh, sv, core, j == 0);
+                            mma_commit(&bars->o_bar[hh]);
+                        }
+                        if (!ok) break;
                         mma_commit(&bars->v_empty[sv]);
                         ++vc;
                     }
-                    return true;
-                };
-                for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
-                    const bool core = tile_is_core(G, j);
-                    const uint32_t s = kc % C::KST;
-                    if (!(ok = lane_wait(&bars->k_full[s], (kc / C::KST) & 1, bars))) break;
-                    for (int hh = 0; hh < 2; ++hh) {
-                        // S is free once its previous occupant has been read:
-                        // half B's previous tile before S_A, half A's current
-                        // tile before S_B.
-                        if (hh == 1 || it > 0) {
-                            const uint32_t prev = hh == 0 ? it - 1 : it;
-                            if (!(ok = lane_wait(&bars->s_free[hh ^ 1], prev & 1, bars))) break;
-                        }
-                        if (core && j == G.n_local &&
-                            !(ok = lane_wait(&bars->qh_full[hh], cq & 1, bars)))
-                            break;
-                        tc_fence_after_sync();
-                        qk(hh, s, core);
-                        mma_commit(&bars->s_full[hh]);
-                        if (hh == 1) {
-                            mma_commit(&bars->k_empty[s]);
-                            ++kc;
-                            if (j == G.n_tiles - 1) mma_commit(&bars->q_empty);
-                        }
-                        if (j > 0 && !(ok = issue_pv(hh, j - 1))) break;
-                    }
                 }
-                if (ok) ok = issue_pv(0, G.n_tiles - 1) && issue_pv(1, G.n_tiles - 1);
-                if (core_block) ++cq;
+                // Wait for every P V this thread issued to finish.
+                mma_commit(&bars->mma_done2);
+                wait_bounded(&bars->mma_done2, 0, &bars->never, kWaitLimitNs);
             }
-            // Wait for every issued tensor-core operation to finish.
-            mma_commit(&bars->mma_done);
-            wait_bounded(&bars->mma_done, 0, &bars->never, kWaitLimitNs);
         }
     } else if (warp < 8) {
         // ------------------------------------------------ softmax warps

@@ -62,6 +62,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return done != 0;
 }
 
+// Non-blocking test of the same condition.  Measured on B200, a thread
+// that issues tensor-core MMAs loses less time on a completed barrier with
+// this test than with try_wait.
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(done)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
 // Wait until the phase of `bar` with the given parity has completed, for at
 // most `limit_ns` nanoseconds.  Returns false if the wait ran out or if
 // `*abort` became nonzero (another role of the CTA gave up).
@@ -69,7 +85,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t *bar, uint32_t parity,
                                              const volatile int *abort,
                                              uint64_t limit_ns)
 {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_test_wait(bar, parity)) return true;
     const uint64_t start = global_timer_ns();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
