@@ -533,17 +533,13 @@ __global__ void __launch_bounds__(352, 1)
                     m_run = m_tile;
                 }
                 const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-                // P V of the previous tile (over all items) must have read
-                // P_h and written O_h before either is touched.  Waiting here
-                // lets each chunk of P go to tensor memory as soon as it is
-                // computed; holding all of P in registers until after the
-                // exponentials spills registers and measured 4% slower on
-                // B200 at 128K context.
-                if (it > 0) {
-                    if (!(ok = warp_wait(&bars->o_bar[hh], (it - 1) & 1, bars))) break;
-                    tc_fence_after_sync();
-                }
-                // P = 2^(S c - m), packed and written chunk by chunk
+                // P = 2^(S c - m), packed.  P V of the previous tile (over
+                // all items) must have read P_h and written O_h before
+                // either is touched: the wait comes after three of the four
+                // chunks, when that P V has almost always finished, and the
+                // last chunk goes to tensor memory as soon as it is computed.
+                // Measured on B200 at 128K context, waiting before the first
+                // chunk is 7% slower, after the first 3% slower.
                 const float2 c2 = make_float2(p.scale_log2, p.scale_log2);
                 const float2 nm2 = make_float2(-m_use, -m_use);
                 float2 acc = make_float2(0.f, 0.f);
@@ -557,8 +553,18 @@ __global__ void __launch_bounds__(352, 1)
                         exp_chunk<true>(xc, c2, nm2, pk[c], acc);
                     else
                         exp_chunk<false>(xc, c2, nm2, pk[c], acc);
-                    tmem_st16(p_addr + c * 16, pk[c]);
+                    if (c == 2) {
+                        if (it > 0) {
+                            if (!(ok = warp_wait(&bars->o_bar[hh], (it - 1) & 1, bars))) break;
+                            tc_fence_after_sync();
+                        }
+#pragma unroll
+                        for (int q = 0; q < 3; ++q) tmem_st16(p_addr + q * 16, pk[q]);
+                    } else if (c >= 3) {
+                        tmem_st16(p_addr + c * 16, pk[c]);
+                    }
                 }
+                if (!ok) break;
                 l_run = fmaf(l_run, alpha, acc.x + acc.y);
                 // the max moved (rare): rescale O before P V of this tile
                 if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
