@@ -164,6 +164,36 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                            cca_dtype o_dtype, void *workspace,
                            size_t workspace_bytes, cudaStream_t stream);
 
+/*
+ * Per-row lengths in device memory.  These two calls read each batch row's
+ * length from `lens` (device memory, B entries of long long, 8-byte
+ * aligned) instead of c->len, so rows may have different lengths and a
+ * sequence of decode steps can be captured once in a CUDA graph and
+ * replayed (nothing the host must know changes from step to step).
+ * c->len is neither read nor written.
+ *
+ * cca_cache_append_rows: row b appends its token t = lens[b] exactly as
+ * cca_cache_append does (ring slot t % tail_cap, pooling of group t / g when
+ * the token completes it), then sets lens[b] = t + 1, all on the device.  A
+ * row whose token would not fit (t / g >= core_cap) is left unchanged and
+ * cca_device_status() reports CCA_ERR_CAPACITY.  Requires Hkv <= 32 (one
+ * warp per key/value head in one block per row): CCA_ERR_UNSUPPORTED
+ * otherwise.
+ */
+cca_status cca_cache_append_rows(const cca_cache *c, long long *lens, const void *q_t,
+                                 const void *k_t, const void *v_t, cudaStream_t stream);
+
+/*
+ * cca_attn_decode_rows: cca_attn_decode for token t_b = lens[b] - 1 of
+ * every row b, each over its own core slots and ring window.  The workspace
+ * is the same as cca_attn_decode's.  A row with lens[b] == 0 gets a zero
+ * output; a row longer than the cache gets a zero output and
+ * cca_device_status() reports CCA_ERR_CAPACITY.
+ */
+cca_status cca_attn_decode_rows(const cca_cache *c, const long long *lens, const void *q_t,
+                                void *o_t, cca_dtype o_dtype, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
 /* Size of the library's fixed decode scratch (bytes): the largest
  * cca_decode_workspace_bytes() that cca_attn_decode_noalloc can serve. */
 #define CCA_NOALLOC_SCRATCH_BYTES (4u << 20)
@@ -191,10 +221,23 @@ cca_status cca_attn_decode_noalloc(const cca_cache *c, const void *q_t, void *o_
 /*
  * Synchronise `stream`, then report CCA_ERR_CUDA if a CUDA error is
  * pending, CCA_ERR_TIMEOUT if any kernel of this library recorded a
- * timed-out wait since the last call, CCA_ERR_RANGE if one clamped a value
- * to the fp16 range, else CCA_OK.  The records are cleared.
+ * timed-out wait since the last call, CCA_ERR_CAPACITY if a per-row call
+ * met a row longer than its cache, CCA_ERR_RANGE if one clamped a value to
+ * the fp16 range, else CCA_OK.  The records are cleared.
  */
 cca_status cca_device_status(cudaStream_t stream);
+
+/*
+ * Failure-path self-test: launch on `stream` one small kernel that waits,
+ * with the library's bounded wait and a limit of `limit_us` microseconds
+ * (1 .. 2000000), on a barrier that nothing completes.  The wait runs out
+ * and the kernel records a timeout, so a later cca_device_status(stream)
+ * returns CCA_ERR_TIMEOUT, and the context stays usable (no fault, trap or
+ * hang).  The pages define no such step; it lets callers and tests check
+ * how the library reports a stuck kernel.  CCA_ERR_INVALID_ARG for a limit
+ * outside the range (nothing launched), CCA_ERR_CUDA on a launch error.
+ */
+cca_status cca_selftest_wait_timeout(unsigned int limit_us, cudaStream_t stream);
 
 /* Human-readable name of a status. */
 const char *cca_status_string(cca_status s);

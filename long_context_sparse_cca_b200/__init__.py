@@ -10,7 +10,9 @@ Build the library with ``python -m long_context_sparse_cca_b200.build``.
 
 Entry points (same names as the C ABI):
     cca_pool, cca_attn_prefill, cca_cache_prefill, cca_cache_append,
-    cca_attn_decode, cca_decode_workspace_bytes, cca_device_status
+    cca_attn_decode, cca_decode_workspace_bytes, cca_attn_decode_noalloc,
+    cca_cache_append_rows, cca_attn_decode_rows (per-row lengths in device
+    memory), cca_selftest_wait_timeout, cca_device_status
 and the ``Cache`` class holding a decode cache's device buffers.
 """
 
@@ -39,7 +41,8 @@ NOALLOC_SCRATCH_BYTES = 4 << 20  # CCA_NOALLOC_SCRATCH_BYTES of include/cca.h
 EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
            "cca_device_status", "cca_status_string", "cca_version", "cca_last_error",
-           "cca_attn_decode_noalloc")
+           "cca_attn_decode_noalloc", "cca_selftest_wait_timeout",
+           "cca_cache_append_rows", "cca_attn_decode_rows")
 
 
 class CCAError(RuntimeError):
@@ -88,6 +91,12 @@ def lib():
     L.cca_attn_decode.restype = st
     L.cca_attn_decode_noalloc.argtypes = [CP, P, P, i, P]
     L.cca_attn_decode_noalloc.restype = st
+    L.cca_cache_append_rows.argtypes = [CP, P, P, P, P, P]
+    L.cca_cache_append_rows.restype = st
+    L.cca_attn_decode_rows.argtypes = [CP, P, P, P, i, P, ctypes.c_size_t, P]
+    L.cca_attn_decode_rows.restype = st
+    L.cca_selftest_wait_timeout.argtypes = [ctypes.c_uint, P]
+    L.cca_selftest_wait_timeout.restype = st
     L.cca_device_status.argtypes = [P]
     L.cca_device_status.restype = st
     L.cca_status_string.argtypes = [i]
@@ -222,6 +231,21 @@ class Cache:
                                    B, Hq, Hkv, d, g, w, core_cap, tail_cap, 0)
         self.workspace = None
 
+    def row(self, b: int) -> "Cache":
+        """Row b alone: a B = 1 cache over the same device buffers (for
+        example to fill rows from prefixes of different lengths with
+        cca_cache_prefill before decoding them with per-row lengths)."""
+        v = object.__new__(Cache)
+        v.k_core, v.v_core = self.k_core[b:b + 1], self.v_core[b:b + 1]
+        v.k_tail, v.v_tail = self.k_tail[b:b + 1], self.v_tail[b:b + 1]
+        st = self.struct
+        v.struct = _CacheStruct(v.k_core.data_ptr(), v.v_core.data_ptr(),
+                                v.k_tail.data_ptr(), v.v_tail.data_ptr(),
+                                1, st.Hq, st.Hkv, st.d, st.g, st.w, st.core_cap,
+                                st.tail_cap, 0)
+        v.workspace = None
+        return v
+
     @property
     def len(self) -> int:
         return int(self.struct.len)
@@ -280,6 +304,48 @@ def cca_attn_decode(cache: Cache, q_t, o_t=None, out_dtype=None,
     return o_t
 
 
+def _lens(lens):
+    torch = _torch()
+    if not (isinstance(lens, torch.Tensor) and lens.is_cuda and lens.dtype == torch.int64
+            and lens.is_contiguous()):
+        raise ValueError("lens must be a contiguous int64 CUDA tensor of B entries")
+    return ctypes.c_void_p(lens.data_ptr())
+
+
+def cca_cache_append_rows(cache: Cache, lens, q_t, k_t, v_t, stream=None) -> None:
+    """Append one token per row, row b at position lens[b]; lens (int64,
+    CUDA, [B]) is advanced on the device.  cache.len is not used."""
+    if lens.numel() != cache.B:
+        raise ValueError("lens needs one entry per batch row")
+    _check(lib().cca_cache_append_rows(ctypes.byref(cache.struct), _lens(lens),
+                                       _dev(q_t, "q_t"), _dev(k_t, "k_t"), _dev(v_t, "v_t"),
+                                       _stream(stream)), "cca_cache_append_rows")
+
+
+def cca_attn_decode_rows(cache: Cache, lens, q_t, o_t=None, out_dtype=None,
+                         workspace=None, stream=None):
+    """Attention of token lens[b] - 1 of every row b (lens: int64, CUDA, [B]):
+    q_t [B,Hq,d] -> o_t [B,Hq,d].  Capturable in a CUDA graph."""
+    torch = _torch()
+    if lens.numel() != cache.B:
+        raise ValueError("lens needs one entry per batch row")
+    if o_t is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
+    od = _odtype(o_t.dtype)
+    nbytes = cca_decode_workspace_bytes(cache)
+    if workspace is None:
+        if cache.workspace is None or cache.workspace.numel() < nbytes:
+            cache.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8,
+                                          device=q_t.device)
+        workspace = cache.workspace
+    _check(lib().cca_attn_decode_rows(
+        ctypes.byref(cache.struct), _lens(lens), _dev(q_t, "q_t"),
+        _dev(o_t, "o_t", o_t.dtype), od, ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel(), _stream(stream)), "cca_attn_decode_rows")
+    return o_t
+
+
 def cca_attn_decode_noalloc(cache: Cache, q_t, o_t=None, out_dtype=None, stream=None):
     """As cca_attn_decode, with the library's fixed device scratch in place
     of a workspace (for callers that cannot allocate device memory)."""
@@ -292,6 +358,14 @@ def cca_attn_decode_noalloc(cache: Cache, q_t, o_t=None, out_dtype=None, stream=
         ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(o_t, "o_t", o_t.dtype), od,
         _stream(stream)), "cca_attn_decode_noalloc")
     return o_t
+
+
+def cca_selftest_wait_timeout(limit_us: int = 1000, stream=None) -> None:
+    """Launch the failure-path self-test kernel: a bounded wait on a barrier
+    that nothing completes.  cca_device_status() afterwards returns
+    CCA_ERR_TIMEOUT; the context stays usable."""
+    _check(lib().cca_selftest_wait_timeout(int(limit_us), _stream(stream)),
+           "cca_selftest_wait_timeout")
 
 
 def cca_device_status(stream=None) -> int:

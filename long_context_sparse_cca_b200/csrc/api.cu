@@ -185,17 +185,56 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                                         c->tail_cap, t, stream));
 }
 
+cca_status cca_cache_append_rows(const cca_cache *c, long long *lens, const void *q_t,
+                                 const void *k_t, const void *v_t, cudaStream_t stream)
+{
+    const cca_status s = cache_status(c);
+    if (s != CCA_OK) return s;
+    if (!ptr_ok(q_t, true) || !ptr_ok(k_t, true) || !ptr_ok(v_t, true) ||
+        lens == nullptr || (reinterpret_cast<uintptr_t>(lens) & 7u) != 0)
+        return CCA_ERR_INVALID_ARG;
+    // one CTA per row, one warp per key/value head
+    if (c->Hkv > 32 || cca::append_rows_smem_bytes(c->Hq, c->Hkv, c->g) > 200u * 1024u)
+        return CCA_ERR_UNSUPPORTED;
+    return from_cuda(cca::launch_append_rows(q_t, k_t, v_t, c->k_core, c->v_core, c->k_tail,
+                                             c->v_tail, lens, c->B, c->Hq, c->Hkv, c->d,
+                                             c->g, c->core_cap, c->tail_cap, stream));
+}
+
+cca_status cca_attn_decode_rows(const cca_cache *c, const long long *lens, const void *q_t,
+                                void *o_t, cca_dtype o_dtype, void *workspace,
+                                size_t workspace_bytes, cudaStream_t stream)
+{
+    const cca_status s = cache_status(c);
+    if (s != CCA_OK) return s;
+    if (o_dtype != CCA_BF16 && o_dtype != CCA_F32) return CCA_ERR_INVALID_ARG;
+    if (!ptr_ok(q_t, true) || !ptr_ok(o_t, true) || workspace == nullptr ||
+        (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 || lens == nullptr ||
+        (reinterpret_cast<uintptr_t>(lens) & 7u) != 0)
+        return CCA_ERR_INVALID_ARG;
+    if (workspace_bytes < cca::decode_workspace_bytes(c->B, c->Hq, c->Hkv, c->d, c->core_cap,
+                                                      c->tail_cap))
+        return CCA_ERR_INVALID_ARG;
+    return from_cuda(cca::launch_decode_rows(c->k_core, c->v_core, c->k_tail, c->v_tail, q_t,
+                                             o_t, o_dtype == CCA_F32, workspace, lens, c->B,
+                                             c->Hq, c->Hkv, c->d, c->g, c->w, c->core_cap,
+                                             c->tail_cap, stream));
+}
+
 cca_status cca_device_status(cudaStream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int a = 0, b = 0, c = 0;
+    unsigned int a = 0, b = 0, c = 0, d = 0, f = 0;
     if ((e = cca::prefill_status_read_clear(&a)) != cudaSuccess ||
         (e = cca::pool_status_read_clear(&b)) != cudaSuccess ||
-        (e = cca::append_status_read_clear(&c)) != cudaSuccess)
+        (e = cca::append_status_read_clear(&c)) != cudaSuccess ||
+        (e = cca::selftest_status_read_clear(&d)) != cudaSuccess ||
+        (e = cca::decode_status_read_clear(&f)) != cudaSuccess)
         return from_cuda(e);
-    const unsigned int st = a | b | c;
+    const unsigned int st = a | b | c | d | f;
     if (st & cca::kStatusTimeout) return CCA_ERR_TIMEOUT;
+    if (st & cca::kStatusCapacity) return CCA_ERR_CAPACITY;
     if (st & cca::kStatusRange) return CCA_ERR_RANGE;
     return CCA_OK;
 }

@@ -12,7 +12,7 @@
 
 namespace cca {
 
-__device__ unsigned int g_append_status;  // kStatusRange: a core value was clamped
+__device__ unsigned int g_append_status;  // kStatusRange, kStatusCapacity
 
 namespace {
 
@@ -39,21 +39,19 @@ __global__ void tail_fill_kernel(const uint4 *__restrict__ K,
 
 constexpr int kAppendWarps = 4;
 
-// One warp per (batch, key/value head).
+// Append token t of pair bh = b * Hkv + h: its ring slot, and if it is the
+// last token of group t / g, the pooling of that group into core slot t / g
+// (the group's older tokens come from the ring, this one from the input
+// rows).  One warp.
 template <int D>
-__global__ void __launch_bounds__(kAppendWarps * 32)
-    append_kernel(const uint16_t *__restrict__ q_t,
-                  const uint16_t *__restrict__ k_t,
-                  const uint16_t *__restrict__ v_t, uint16_t *__restrict__ k_core,
-                  uint16_t *__restrict__ v_core, uint16_t *__restrict__ k_tail,
-                  uint16_t *__restrict__ v_tail, int B, int Hq, int Hkv, int g,
-                  int64_t core_cap, int64_t tail_cap, int64_t t, int do_pool,
-                  float scale_log2)
+__device__ __forceinline__ void append_pair(
+    const uint16_t *__restrict__ q_t, const uint16_t *__restrict__ k_t,
+    const uint16_t *__restrict__ v_t, uint16_t *__restrict__ k_core,
+    uint16_t *__restrict__ v_core, uint16_t *__restrict__ k_tail,
+    uint16_t *__restrict__ v_tail, int Hq, int Hkv, int g, int64_t core_cap,
+    int64_t tail_cap, int64_t t, int64_t bh, float scale_log2, float *scratch)
 {
-    extern __shared__ float append_smem[];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t bh = static_cast<int64_t>(blockIdx.x) * kAppendWarps + warp;
-    if (bh >= static_cast<int64_t>(B) * Hkv) return;
+    const int lane = threadIdx.x & 31;
     const int r = Hq / Hkv;
     const int64_t b = bh / Hkv, h = bh - b * Hkv;
     using VT = typename RowVec<D>::T;
@@ -62,13 +60,10 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
     const int64_t slot = t % tail_cap;
     reinterpret_cast<VT *>(k_tail + (bh * tail_cap + slot) * D)[lane] = kin[lane];
     reinterpret_cast<VT *>(v_tail + (bh * tail_cap + slot) * D)[lane] = vin[lane];
-    if (!do_pool) return;
-    // The group's older tokens come from the ring; its newest one (this
-    // token) is read from the input rows.
+    if ((t + 1) % g != 0) return;
     const int64_t first = t - g + 1, j = t / g;
     const uint16_t *kt_base = k_tail + bh * tail_cap * D;
     const uint16_t *vt_base = v_tail + bh * tail_cap * D;
-    float *scratch = append_smem + warp * (r * g + g);
     const bool over = pool_group_warp<D>(
         [&](int i) {
             return i == g - 1 ? k_t + bh * D
@@ -81,6 +76,56 @@ __global__ void __launch_bounds__(kAppendWarps * 32)
         [&](int k) { return q_t + (b * Hq + h * r + k) * D; }, r, g, scale_log2,
         scratch, k_core + (bh * core_cap + j) * D, v_core + (bh * core_cap + j) * D);
     if (over && lane == 0) atomicOr(&g_append_status, kStatusRange);
+}
+
+// One warp per (batch, key/value head); every row appends token t.
+template <int D>
+__global__ void __launch_bounds__(kAppendWarps * 32)
+    append_kernel(const uint16_t *__restrict__ q_t,
+                  const uint16_t *__restrict__ k_t,
+                  const uint16_t *__restrict__ v_t, uint16_t *__restrict__ k_core,
+                  uint16_t *__restrict__ v_core, uint16_t *__restrict__ k_tail,
+                  uint16_t *__restrict__ v_tail, int B, int Hq, int Hkv, int g,
+                  int64_t core_cap, int64_t tail_cap, int64_t t, float scale_log2)
+{
+    extern __shared__ float append_smem[];
+    const int warp = threadIdx.x >> 5;
+    const int64_t bh = static_cast<int64_t>(blockIdx.x) * kAppendWarps + warp;
+    if (bh >= static_cast<int64_t>(B) * Hkv) return;
+    const int r = Hq / Hkv;
+    append_pair<D>(q_t, k_t, v_t, k_core, v_core, k_tail, v_tail, Hq, Hkv, g, core_cap,
+                   tail_cap, t, bh, scale_log2, append_smem + warp * (r * g + g));
+}
+
+// One CTA per batch row b, one warp per key/value head; row b appends its
+// token lens[b] and then advances lens[b] (device memory, so a captured
+// CUDA graph can replay decode steps).  A row whose token would not fit the
+// cache is left unchanged and reported (kStatusCapacity).
+template <int D>
+__global__ void append_rows_kernel(const uint16_t *__restrict__ q_t,
+                                   const uint16_t *__restrict__ k_t,
+                                   const uint16_t *__restrict__ v_t,
+                                   uint16_t *__restrict__ k_core, uint16_t *__restrict__ v_core,
+                                   uint16_t *__restrict__ k_tail, uint16_t *__restrict__ v_tail,
+                                   long long *__restrict__ lens, int Hq, int Hkv, int g,
+                                   int64_t core_cap, int64_t tail_cap, float scale_log2)
+{
+    extern __shared__ float append_smem[];
+    __shared__ long long row_len;
+    const int warp = threadIdx.x >> 5;
+    const int64_t b = blockIdx.x;
+    if (threadIdx.x == 0) row_len = lens[b];
+    __syncthreads();
+    const int64_t t = row_len;
+    if (t < 0 || t / g >= core_cap) {
+        if (threadIdx.x == 0) atomicOr(&g_append_status, kStatusCapacity);
+        return;
+    }
+    const int r = Hq / Hkv;
+    append_pair<D>(q_t, k_t, v_t, k_core, v_core, k_tail, v_tail, Hq, Hkv, g, core_cap,
+                   tail_cap, t, b * Hkv + warp, scale_log2, append_smem + warp * (r * g + g));
+    __syncthreads();  // every warp has read row_len before it moves on
+    if (threadIdx.x == 0) lens[b] = t + 1;
 }
 
 }  // namespace
@@ -112,7 +157,6 @@ cudaError_t launch_append(const void *q_t, const void *k_t, const void *v_t,
     const int blocks = static_cast<int>((pairs + kAppendWarps - 1) / kAppendWarps);
     const int r = Hq / Hkv;
     const size_t smem = sizeof(float) * kAppendWarps * (r * g + g);
-    const int do_pool = ((t + 1) % g) == 0;
     const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
     auto args = [&](auto kern) {
         if (smem > 48 * 1024)
@@ -123,13 +167,44 @@ cudaError_t launch_append(const void *q_t, const void *k_t, const void *v_t,
             static_cast<const uint16_t *>(v_t), static_cast<uint16_t *>(k_core),
             static_cast<uint16_t *>(v_core), static_cast<uint16_t *>(k_tail),
             static_cast<uint16_t *>(v_tail), B, Hq, Hkv, g, core_cap, tail_cap, t,
-            do_pool, scale_log2);
+            scale_log2);
     };
     if (d == 128)
         args(append_kernel<128>);
     else
         args(append_kernel<64>);
     return cudaGetLastError();
+}
+
+cudaError_t launch_append_rows(const void *q_t, const void *k_t, const void *v_t,
+                               void *k_core, void *v_core, void *k_tail, void *v_tail,
+                               long long *lens, int B, int Hq, int Hkv, int d, int g,
+                               int64_t core_cap, int64_t tail_cap, cudaStream_t s)
+{
+    const int r = Hq / Hkv;
+    const size_t smem = sizeof(float) * Hkv * (r * g + g);
+    const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+    auto args = [&](auto kern) {
+        if (smem > 48 * 1024)
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+        kern<<<B, Hkv * 32, smem, s>>>(
+            static_cast<const uint16_t *>(q_t), static_cast<const uint16_t *>(k_t),
+            static_cast<const uint16_t *>(v_t), static_cast<uint16_t *>(k_core),
+            static_cast<uint16_t *>(v_core), static_cast<uint16_t *>(k_tail),
+            static_cast<uint16_t *>(v_tail), lens, Hq, Hkv, g, core_cap, tail_cap,
+            scale_log2);
+    };
+    if (d == 128)
+        args(append_rows_kernel<128>);
+    else
+        args(append_rows_kernel<64>);
+    return cudaGetLastError();
+}
+
+size_t append_rows_smem_bytes(int Hq, int Hkv, int g)
+{
+    return sizeof(float) * Hkv * ((Hq / Hkv) * g + g);
 }
 
 cudaError_t append_status_read_clear(unsigned int *v)

@@ -61,6 +61,7 @@ __device__ __forceinline__ float f16_hi(uint32_t v)
 constexpr float kF16Max = 65504.0f;
 constexpr unsigned int kStatusTimeout = 1u;  // a bounded wait ran out
 constexpr unsigned int kStatusRange = 2u;    // a value exceeded the fp16 range
+constexpr unsigned int kStatusCapacity = 4u; // a row's length exceeded the cache
 
 __device__ __forceinline__ float clamp_f16(float x, bool &over)
 {

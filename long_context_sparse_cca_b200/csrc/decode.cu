@@ -16,6 +16,8 @@
 
 namespace cca {
 
+__device__ unsigned int g_decode_status;  // kStatusCapacity
+
 namespace {
 
 constexpr int kDecodeThreads = 128;
@@ -72,7 +74,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         float *__restrict__ part_o, float2 *__restrict__ part_ml,
                         unsigned int *__restrict__ tickets, void *__restrict__ o_t,
                         int out_f32, int Hq, int Hkv, int64_t n_keys, int chunk,
-                        int nsplit, float scale_log2)
+                        int nsplit, float scale_log2, const long long *__restrict__ lens,
+                        int g, int w, int64_t core_cap, int stride)
 {
     using S = DecodeShape<D>;
     extern __shared__ float dsm[];
@@ -85,6 +88,35 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int64_t b = bh / Hkv, h = bh - b * Hkv;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int kl = lane % S::KL, kg = warp * S::KPW + lane / S::KL;
+    // Uniform lengths: the host planned the split.  Per-row lengths (lens
+    // in device memory): this CTA plans its own row; the grid covers the
+    // cache's capacity and CTAs past the row's keys leave at once.
+    CacheView cvb = cv;
+    if (lens != nullptr) {
+        const int64_t tb = lens[b] - 1;
+        const int64_t wsb = tb >= 0 ? window_start(tb, g, w) : 0;
+        if (tb < 0 || wsb / g > core_cap) {
+            // an empty row has zero output; a row past the cache is reported
+            if (split == 0) {
+                if (tb >= 0 && tid == 0) atomicOr(&g_decode_status, kStatusCapacity);
+                for (int idx = tid; idx < r * D; idx += kDecodeThreads) {
+                    const int64_t orow = b * Hq + h * r + idx / D;
+                    if (out_f32)
+                        static_cast<float *>(o_t)[orow * D + idx % D] = 0.f;
+                    else
+                        static_cast<uint16_t *>(o_t)[orow * D + idx % D] = 0;
+                }
+            }
+            return;
+        }
+        cvb.ws = wsb;
+        cvb.n_core = wsb / g;
+        n_keys = cvb.n_core + (tb - wsb + 1);
+        nsplit = static_cast<int>((n_keys + chunk - 1) / chunk);
+        if (split >= nsplit) return;
+    } else {
+        stride = nsplit;
+    }
     const int64_t c0 = static_cast<int64_t>(split) * chunk;
     const int64_t c1 = c0 + chunk < n_keys ? c0 + chunk : n_keys;
     const int nk = static_cast<int>(c1 - c0);
@@ -112,7 +144,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             kv[u] = make_uint4(0u, 0u, 0u, 0u);
             kcore[u] = false;
             if (i < nk) {
-                const int64_t row = cv.row(bh, c0 + i, kcore[u]);
+                const int64_t row = cvb.row(bh, c0 + i, kcore[u]);
                 const uint16_t *src = kcore[u] ? cv.k_core : cv.k_tail;
                 kv[u] = ldg_stream(src + row * D + kl * 8);
             }
@@ -173,7 +205,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             vv[u] = make_uint4(0u, 0u, 0u, 0u);
             vcore[u] = false;
             if (i < nk) {
-                const int64_t row = cv.row(bh, c0 + i, vcore[u]);
+                const int64_t row = cvb.row(bh, c0 + i, vcore[u]);
                 const uint16_t *src = vcore[u] ? cv.v_core : cv.v_tail;
                 vv[u] = ldg_stream(src + row * D + kl * 8);
             }
@@ -206,7 +238,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
         float s = 0.f;
 #pragma unroll 4
         for (int gi = 0; gi < S::NG; ++gi) s += red[(gi * R + k) * D + c];
-        const int64_t qrow = (b * Hq + h * r + k) * nsplit + split;
+        const int64_t qrow = (b * Hq + h * r + k) * stride + split;
         part_o[qrow * D + c] = s;
         if (c == 0) part_ml[qrow] = make_float2(stat[2 * k], stat[2 * k + 1]);
     }
@@ -228,7 +260,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     // several independent 16-byte loads of partial outputs in flight.
     const bool wfit = nsplit <= chunk;
     for (int k = warp; k < r; k += kDecodeThreads / 32) {
-        const float2 *ml = part_ml + (b * Hq + h * r + k) * nsplit;
+        const float2 *ml = part_ml + (b * Hq + h * r + k) * stride;
         float mx = -INFINITY;
         for (int sp = lane; sp < nsplit; sp += 32) mx = fmaxf(mx, __ldcg(&ml[sp].x));
         mx = warp_max(mx);
@@ -252,8 +284,8 @@ __global__ void __launch_bounds__(kDecodeThreads)
     const int c4 = tid % C4, g0 = tid / C4;
     for (int k = 0; k < r; ++k) {
         const int64_t orow = b * Hq + h * r + k;
-        const float2 *ml = part_ml + orow * nsplit;
-        const float4 *po4 = reinterpret_cast<const float4 *>(part_o + orow * nsplit * D) + c4;
+        const float2 *ml = part_ml + orow * stride;
+        const float4 *po4 = reinterpret_cast<const float4 *>(part_o + orow * stride * D) + c4;
         const float mx = stat[2 * k];
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
@@ -295,7 +327,8 @@ template <int D, int R>
 cudaError_t launch_split(const CacheView &cv, const void *q_t, float *part_o,
                          float2 *part_ml, unsigned int *tickets, void *o_t, bool o_f32,
                          int B, int Hq, int Hkv, int64_t n_keys, int nsplit,
-                         float scale_log2, cudaStream_t s)
+                         float scale_log2, cudaStream_t s, const long long *lens = nullptr,
+                         int g = 0, int w = 0, int64_t core_cap = 0, int stride = 0)
 {
     using S = DecodeShape<D>;
     const size_t smem =
@@ -308,7 +341,7 @@ cudaError_t launch_split(const CacheView &cv, const void *q_t, float *part_o,
     kern<<<grid, kDecodeThreads, smem, s>>>(cv, static_cast<const uint16_t *>(q_t),
                                             part_o, part_ml, tickets, o_t, o_f32 ? 1 : 0,
                                             Hq, Hkv, n_keys, kDecodeChunk, nsplit,
-                                            scale_log2);
+                                            scale_log2, lens, g, w, core_cap, stride);
     return cudaGetLastError();
 }
 
@@ -400,6 +433,60 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
         else CCA_SPLIT(64, 16);
     }
 #undef CCA_SPLIT
+    return e;
+}
+
+cudaError_t launch_decode_rows(const void *k_core, const void *v_core,
+                               const void *k_tail, const void *v_tail,
+                               const void *q_t, void *o_t, bool o_f32,
+                               void *workspace, const long long *lens, int B, int Hq,
+                               int Hkv, int d, int g, int w, int64_t core_cap,
+                               int64_t tail_cap, cudaStream_t s)
+{
+    const WorkspaceLayout L = workspace_layout(B, Hq, Hkv, d, core_cap, tail_cap);
+    const int maxs = decode_max_splits(core_cap, tail_cap);
+    char *ws = static_cast<char *>(workspace);
+    float *part_o = reinterpret_cast<float *>(ws);
+    float2 *part_ml = reinterpret_cast<float2 *>(ws + L.o_bytes);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + L.o_bytes + L.ml_bytes);
+    // ws and n_core are planned per row inside the kernel
+    CacheView cv{static_cast<const uint16_t *>(k_core),
+                 static_cast<const uint16_t *>(v_core),
+                 static_cast<const uint16_t *>(k_tail),
+                 static_cast<const uint16_t *>(v_tail),
+                 core_cap,
+                 tail_cap,
+                 0,
+                 0};
+    const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+    const int r = Hq / Hkv;
+    cudaError_t e = cudaMemsetAsync(tickets, 0, sizeof(unsigned int) * B * Hkv, s);
+    if (e != cudaSuccess) return e;
+#define CCA_SPLIT(DD, RR)                                                            \
+    e = launch_split<DD, RR>(cv, q_t, part_o, part_ml, tickets, o_t, o_f32, B, Hq,   \
+                             Hkv, 0, maxs, scale_log2, s, lens, g, w, core_cap, maxs)
+    if (d == 128) {
+        if (r == 1) CCA_SPLIT(128, 1);
+        else if (r == 2) CCA_SPLIT(128, 2);
+        else if (r <= 4) CCA_SPLIT(128, 4);
+        else if (r <= 8) CCA_SPLIT(128, 8);
+        else CCA_SPLIT(128, 16);
+    } else {
+        if (r == 1) CCA_SPLIT(64, 1);
+        else if (r == 2) CCA_SPLIT(64, 2);
+        else if (r <= 4) CCA_SPLIT(64, 4);
+        else if (r <= 8) CCA_SPLIT(64, 8);
+        else CCA_SPLIT(64, 16);
+    }
+#undef CCA_SPLIT
+    return e;
+}
+
+cudaError_t decode_status_read_clear(unsigned int *v)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(v, g_decode_status, sizeof(*v));
+    if (e == cudaSuccess && *v) e = cudaMemcpyToSymbol(g_decode_status, &zero, sizeof(zero));
     return e;
 }
 

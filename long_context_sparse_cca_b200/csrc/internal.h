@@ -57,6 +57,19 @@ cudaError_t launch_prefill(const void *Q, const void *K, const void *V,
 // Device status words (bits kStatusTimeout, kStatusRange): read and clear.
 cudaError_t prefill_status_read_clear(unsigned int *v);
 cudaError_t pool_status_read_clear(unsigned int *v);
+cudaError_t launch_append_rows(const void *q_t, const void *k_t, const void *v_t,
+                               void *k_core, void *v_core, void *k_tail, void *v_tail,
+                               long long *lens, int B, int Hq, int Hkv, int d, int g,
+                               int64_t core_cap, int64_t tail_cap, cudaStream_t s);
+size_t append_rows_smem_bytes(int Hq, int Hkv, int g);
+cudaError_t launch_decode_rows(const void *k_core, const void *v_core,
+                               const void *k_tail, const void *v_tail,
+                               const void *q_t, void *o_t, bool o_f32,
+                               void *workspace, const long long *lens, int B, int Hq,
+                               int Hkv, int d, int g, int w, int64_t core_cap,
+                               int64_t tail_cap, cudaStream_t s);
 cudaError_t append_status_read_clear(unsigned int *v);
+cudaError_t selftest_status_read_clear(unsigned int *v);
+cudaError_t decode_status_read_clear(unsigned int *v);
 
 }  // namespace cca

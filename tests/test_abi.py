@@ -151,3 +151,9 @@ def test_binding_refuses_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(cca, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="libcca.so not found"):
         cca.lib()
+
+
+def test_selftest_limit_checks(L):
+    # out-of-range limits are refused on the host, before any launch
+    assert L.cca_selftest_wait_timeout(0, None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_selftest_wait_timeout(2000001, None) == cca.CCA_ERR_INVALID_ARG
