@@ -185,6 +185,19 @@ class ClockSampler:
                 "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(values, world: int, device) -> list:
+    """Element-wise maximum of each rank's timings, by one all-reduce over
+    the process group (the identity for a single rank).  Every rank must
+    call it with the same number of values."""
+    if world == 1:
+        return [float(v) for v in values]
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
 # ----------------------------------------------------------------- CUDA arm
 
 def _dev(bits, torch):
@@ -314,18 +327,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         if i > 0:  # first one warms the pinned paths
             e2e_ms.append(a.elapsed_time(b))
 
-    def gather_max(v: float) -> float:
-        if world == 1:
-            return v
-        t = torch.tensor([v], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
-    total_ms = gather_max(total_ms)
-    mean_pool = gather_max(float(np.mean(pool_ms)))
-    mean_prefill = gather_max(float(np.mean(prefill_ms)))
-    mean_decode = gather_max(float(np.mean(decode_ms)))
-    mean_e2e = gather_max(float(np.mean(e2e_ms))) if e2e_ms else None
+    # one all-reduce of every timing, the same on all ranks (no e2e: -1)
+    total_ms, mean_pool, mean_prefill, mean_decode, mean_e2e = max_over_ranks(
+        [total_ms, float(np.mean(pool_ms)), float(np.mean(prefill_ms)),
+         float(np.mean(decode_ms)), float(np.mean(e2e_ms)) if e2e_ms else -1.0],
+        world, "cuda")
+    mean_e2e = mean_e2e if mean_e2e >= 0 else None
     h2d = 3 * Q.numel() * 2 if do_prefill else 0
     d2h = O.numel() * 2 if do_prefill else 0
     return dict(total_ms=total_ms, pool_ms=mean_pool, prefill_ms=mean_prefill,
