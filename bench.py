@@ -383,6 +383,59 @@ def oracle_sample(budget_s: float = 20.0) -> dict:
             "seconds": pool_s + attend_s}
 
 
+def oracle_decode_sample(budget_s: float = 4.0) -> dict:
+    """Time the fp64 oracle's decode step (append + decode) on head 0 of
+    batch row 0 of the decode workload: the cache is built from the
+    65536-token prefix (pooled core slots and the ring), then steps run
+    until the budget or the 256 steps are spent.  Scaled to all rows and
+    heads of the workload."""
+    import dataclasses
+
+    import oracle
+
+    dw = DECODE
+    one = dataclasses.replace(dw, B=1, Hq=1, Hkv=1)  # the same values as head 0 of row 0
+    y = synth.generate(one)
+    q, k, v = (synth.bf16_bits_to_f64(a) for a in (y.q, y.k, y.v))
+    T = dw.T
+    c = oracle.new_cache(1, 1, 1, dw.d, dw.g, dw.w, core_cap=(T + dw.steps) // dw.g)
+    Kc, Vc = oracle.pool(q[:, :, :T], k[:, :, :T], v[:, :, :T], dw.g)
+    m = Kc.shape[2]
+    c.k_core[:, :, :m] = Kc
+    c.v_core[:, :, :m] = Vc
+    cap = c.tail_cap
+    for p in range(T - cap, T):
+        c.k_tail[:, :, p % cap] = k[:, :, p]
+        c.v_tail[:, :, p % cap] = v[:, :, p]
+    c.len = T
+    n = 0
+    t0 = time.perf_counter()
+    while n < dw.steps and (n == 0 or time.perf_counter() - t0 < budget_s):
+        t = T + n
+        c.append(q[:, :, t], k[:, :, t], v[:, :, t])
+        c.decode(q[:, :, t])
+        n += 1
+    sec = time.perf_counter() - t0
+    return {"us_per_step": sec / n * 1e6 * dw.B * dw.Hq, "unit": "us/step",
+            "cores": oracle.threads(), "kind": "oracle",
+            "sample": (f"decode workload, row 0 head 0 of {dw.B} x {dw.Hq}: {n} steps of "
+                       f"append + decode after the 65536-token prefix ({sec:.2f} s); "
+                       "scaled to all rows and heads")}
+
+
+def oracle_single_thread_value(budget_s: float = 3.0) -> float:
+    """The prefill oracle sample on one thread (tokens/s of the full
+    workload), the thread count restored afterwards."""
+    import oracle
+
+    n = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        return oracle_sample(budget_s=budget_s)["value"]
+    finally:
+        oracle.set_threads(n)
+
+
 # ----------------------------------------------------------------- main
 
 def main(argv=None) -> int:
@@ -502,6 +555,8 @@ def main(argv=None) -> int:
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample()
         cb.pop("seconds", None)
+        cb["single_thread_value"] = oracle_single_thread_value()
+        cb["decode"] = oracle_decode_sample()
         line["cpu_baseline"] = cb
     if rank == 0:
         print(json.dumps(line))
