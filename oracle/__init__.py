@@ -2,6 +2,8 @@
 
 A ctypes front end over ``cca_oracle.c`` (fp64, OpenMP), the plain
 restatement of CCA-Attention against which the CUDA library is checked.
+``cca_backward.py`` adds the fp64 gradients (dQ, dK, dV through the fused
+attention and the pooling), pinned to finite differences of the C forward.
 Only the tests, the package's smoke check and the benchmark's CPU-baseline
 leg may import this package; the CUDA library and its Python binding never
 do, and the two share no code.
