@@ -246,6 +246,27 @@ class Cache:
         v.workspace = None
         return v
 
+    def state_dict(self) -> dict:
+        """Host copy of the cache (core slots, ring, shape, length), for
+        saving and later restoring a decode session."""
+        st = self.struct
+        return {"shape": {n: int(getattr(st, n)) for n in
+                          ("B", "Hq", "Hkv", "d", "g", "w", "core_cap", "tail_cap")},
+                "len": int(st.len),
+                "k_core": self.k_core.cpu(), "v_core": self.v_core.cpu(),
+                "k_tail": self.k_tail.cpu(), "v_tail": self.v_tail.cpu()}
+
+    @classmethod
+    def from_state_dict(cls, state: dict, device="cuda") -> "Cache":
+        """A cache on ``device`` holding what ``state_dict`` saved."""
+        sh = state["shape"]
+        c = cls(sh["B"], sh["Hq"], sh["Hkv"], sh["d"], sh["g"], sh["w"], sh["core_cap"],
+                sh["tail_cap"], device=device)
+        for n in ("k_core", "v_core", "k_tail", "v_tail"):
+            getattr(c, n).copy_(state[n])
+        c.len = state["len"]
+        return c
+
     @property
     def len(self) -> int:
         return int(self.struct.len)

@@ -157,3 +157,20 @@ def test_selftest_limit_checks(L):
     # out-of-range limits are refused on the host, before any launch
     assert L.cca_selftest_wait_timeout(0, None) == cca.CCA_ERR_INVALID_ARG
     assert L.cca_selftest_wait_timeout(2000001, None) == cca.CCA_ERR_INVALID_ARG
+
+
+def test_cache_state_round_trip():
+    # save/restore of a decode session is a host copy of the caller-owned
+    # buffers plus the length (tensors on the CPU here; no kernel runs)
+    import torch
+    c = cca.Cache(2, 4, 2, 64, 16, 32, core_cap=8, device="cpu")
+    for t in (c.k_core, c.v_core, c.k_tail, c.v_tail):
+        t.copy_(torch.randn(t.shape).to(t.dtype))
+    c.len = 77
+    st = c.state_dict()
+    d = cca.Cache.from_state_dict(st, device="cpu")
+    assert d.len == 77 and (d.B, d.Hq, d.Hkv, d.d, d.g, d.w, d.core_cap, d.tail_cap) == \
+        (2, 4, 2, 64, 16, 32, 8, 48)
+    for n in ("k_core", "v_core", "k_tail", "v_tail"):
+        assert torch.equal(getattr(c, n), getattr(d, n))
+        assert getattr(d, n).data_ptr() != getattr(c, n).data_ptr()
