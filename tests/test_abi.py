@@ -174,3 +174,42 @@ def test_cache_state_round_trip():
     for n in ("k_core", "v_core", "k_tail", "v_tail"):
         assert torch.equal(getattr(c, n), getattr(d, n))
         assert getattr(d, n).data_ptr() != getattr(c, n).data_ptr()
+
+
+def test_rows_argument_checks(L):
+    """The per-row calls check their arguments on the host, before any
+    launch: every call below fails there."""
+    P = ctypes.c_void_p
+    c = _cache()
+    ws = L.cca_decode_workspace_bytes(ctypes.byref(c))
+    lens = FAKE + (5 << 20)
+    # lens missing or misaligned
+    for bad in (0, lens + 4):
+        assert L.cca_cache_append_rows(ctypes.byref(c), P(bad), P(FAKE), P(FAKE), P(FAKE),
+                                       None) == cca.CCA_ERR_INVALID_ARG
+        assert L.cca_attn_decode_rows(ctypes.byref(c), P(bad), P(FAKE), P(FAKE + 4096), 0,
+                                      P(FAKE), ws, None) == cca.CCA_ERR_INVALID_ARG
+    # invalid cache, output dtype, workspace size and alignment
+    bad = _cache(tail_cap=10)
+    assert L.cca_cache_append_rows(ctypes.byref(bad), P(lens), P(FAKE), P(FAKE), P(FAKE),
+                                   None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_attn_decode_rows(ctypes.byref(c), P(lens), P(FAKE), P(FAKE + 4096), 3,
+                                  P(FAKE), ws, None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_attn_decode_rows(ctypes.byref(c), P(lens), P(FAKE), P(FAKE + 4096), 0,
+                                  P(FAKE), ws - 1, None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_attn_decode_rows(ctypes.byref(c), P(lens), P(FAKE), P(FAKE + 4096), 0,
+                                  P(FAKE + 16), ws, None) == cca.CCA_ERR_INVALID_ARG
+    # one block per row holds one warp per key/value head: at most 32
+    wide = _cache(Hq=64, Hkv=64)
+    assert L.cca_cache_append_rows(ctypes.byref(wide), P(lens), P(FAKE), P(FAKE), P(FAKE),
+                                   None) == cca.CCA_ERR_UNSUPPORTED
+
+
+def test_rows_binding_checks_lens():
+    import torch
+    c = cca.Cache(2, 2, 2, 64, 16, 32, core_cap=4, device="cpu")
+    q = torch.zeros((2, 2, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        cca.cca_cache_append_rows(c, torch.zeros(3, dtype=torch.int64), q, q, q)
+    with pytest.raises(ValueError):
+        cca.cca_attn_decode_rows(c, torch.zeros(2, dtype=torch.int32), q)
