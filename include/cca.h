@@ -41,13 +41,14 @@
  * borrowed for the call; the library allocates nothing.  Calls are
  * asynchronous on the given stream (the CUDA runtime's cudaStream_t; 0 is
  * the legacy default stream).  Outputs must not alias inputs.  Pointers
- * must be 16-byte aligned.
+ * must be 16-byte aligned (the per-row length arrays: 8-byte).
  *
  * Errors: argument checks run on the host before any launch; a call that
  * fails them returns a nonzero status and writes nothing.  CCA_ERR_CUDA
  * reports a launch error.  Device-side waits are bounded: a wait that runs
  * out records a timeout in a device status word and the kernel returns
- * early; cca_device_status() reads and clears it (and the fp16 range flag).
+ * early; cca_device_status() reads and clears it (and the fp16 range and
+ * per-row capacity flags).
  */
 #ifndef CCA_H
 #define CCA_H
