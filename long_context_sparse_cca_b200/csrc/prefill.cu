@@ -57,22 +57,6 @@ namespace {
 
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per wait
 constexpr float kRescaleThreshold = 15.0f;  // log2 units: P stays <= 2^15 (fp16 range)
-// Share of the exponentials computed on the FMA pipe: pairs i with
-// (i % 8) < kPolyPerEight of each 16-pair chunk of a row.  Measured on B200
-// at 128K context against 0/8: 2/8 +7%, 3/8 +8%, 4/8 +11% time (the
-// exponentials run beside the MMAs, so freeing MUFU time gains nothing and
-// the polynomial's extra instructions cost), so it is 0.
-constexpr int kPolyPerEight = 0;
-
-// 2^f on [-1/2, 1/2] by a degree-3 polynomial whose coefficients were fitted
-// for this kernel (Remez exchange on the relative error, weight 2^-f); max
-// relative error 7.5e-5, below half an fp16 spacing (a float32 replay of
-// these steps is checked against 2^y by the tests).
-constexpr float kP0 = 0.9999280571937561f;
-constexpr float kP1 = 0.6932609677314758f;
-constexpr float kP2 = 0.2426111251115799f;
-constexpr float kP3 = 0.0551716685295105f;
-constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23
 
 template <int D>
 struct Pf {
@@ -177,31 +161,11 @@ __device__ __forceinline__ bool lane_wait(uint64_t *bar, uint32_t parity, Bars *
     return ok;
 }
 
-// ------------------------------------------------------------ exp2 on pairs
-
 __device__ __forceinline__ float fmax3(float a, float b, float c)
 {
     float d;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
     return d;
-}
-
-// 2^y for a pair, on the FMA pipe: y = n + f with n = rint(y) read from the
-// low mantissa bits of y + 1.5*2^23, f in [-1/2, 1/2] through the degree-3
-// polynomial, n added to the result's exponent field.  y is clamped to
-// >= -125 first, so the exponent field stays positive (2^-125 is far below
-// anything a row sum can notice; masked logits, -inf, land there).
-__device__ __forceinline__ float2 exp2_poly2(float2 y)
-{
-    y = make_float2(fmaxf(y.x, -125.f), fmaxf(y.y, -125.f));
-    const float2 t = __fadd2_rn(y, make_float2(kRoundMagic, kRoundMagic));
-    const float2 n = __fadd2_rn(t, make_float2(-kRoundMagic, -kRoundMagic));
-    const float2 f = __ffma2_rn(n, make_float2(-1.f, -1.f), y);
-    float2 q = __ffma2_rn(make_float2(kP3, kP3), f, make_float2(kP2, kP2));
-    q = __ffma2_rn(q, f, make_float2(kP1, kP1));
-    q = __ffma2_rn(q, f, make_float2(kP0, kP0));
-    return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                       __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
 }
 
 __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
@@ -212,13 +176,11 @@ __device__ __forceinline__ void load_chunk(uint32_t addr, float (&x)[32])
     for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(u[e]);
 }
 
-// Softmax numerators of one 32-column chunk: p = 2^(x c - m), packed to
-// 16-bit pairs in pk (fp16 for core tiles, bf16 for raw ones).  The MUFU unit computes 16 exponentials
-// per clock per SM, as many as the tile's MMAs need at full rate, so pairs
-// i with (i % 8) < kPolyPerEight take the FMA-pipe polynomial instead.  For
-// bf16 P (8 significant bits) the row sum adds exactly the rounded values
-// P V will see, so that the rounding of a dominant weight cancels in
-// O = (P V) / l; for fp16 P (11 bits) the fp32 values are summed.
+// Softmax numerators of one 32-column chunk: p = 2^(x c - m) on the MUFU
+// unit, packed to 16-bit pairs in pk (fp16 for core tiles, bf16 for raw
+// ones).  For bf16 P (8 significant bits) the row sum adds exactly the
+// rounded values P V will see, so that the rounding of a dominant weight
+// cancels in O = (P V) / l; for fp16 P (11 bits) the fp32 values are summed.
 template <bool F16>
 __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float2 nm2,
                                           uint32_t (&pk)[16], float2 &acc)
@@ -226,9 +188,7 @@ __device__ __forceinline__ void exp_chunk(const float (&x)[32], float2 c2, float
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
         const float2 y = __ffma2_rn(make_float2(x[2 * i], x[2 * i + 1]), c2, nm2);
-        const float2 pv = (i & 7) < kPolyPerEight
-                              ? exp2_poly2(y)
-                              : make_float2(fast_exp2(y.x), fast_exp2(y.y));
+        const float2 pv = make_float2(fast_exp2(y.x), fast_exp2(y.y));
         if (F16) {
             pk[i] = pack_f16x2(pv.x, pv.y);
             acc = __fadd2_rn(acc, pv);

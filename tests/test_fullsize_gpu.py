@@ -10,7 +10,8 @@ oracle computes one by one:
 Pooling is checked in full (every core row); attention on sampled query
 rows (window and group edges, tile edges, the last 64 rows, 256 seeded
 random rows) for every batch entry and head; decode at every step for batch
-row 0 and at 16 sampled steps for all rows.
+row 0 and at 16 sampled steps for all rows, in fp32 and in bf16 (the
+benchmark's output type).
 """
 
 import numpy as np
@@ -79,12 +80,15 @@ def test_decode_64k_256_steps(cca):
     del pre
     nq, nk, nv = (to_cuda(np.ascontiguousarray(a[:, :, wl.T:].transpose(2, 0, 1, 3)))
                   for a in (y.q, y.k, y.v))
-    outs = []
+    outs, outs16 = [], []
     for s in range(wl.steps):
         cca.cca_cache_append(cache, nq[s], nk[s], nv[s])
         outs.append(cca.cca_attn_decode(cache, nq[s], out_dtype=torch.float32))
+        # bf16, as benchmarked
+        outs16.append(cca.cca_attn_decode(cache, nq[s], out_dtype=torch.bfloat16))
     assert cca.cca_device_status() == cca.CCA_OK
     O = torch.stack(outs, dim=2).cpu()  # [B, Hq, steps, d]
+    O16 = torch.stack(outs16, dim=2).cpu()
     m = total // wl.g
     k_core, v_core = cache.k_core[:, :, :m].cpu(), cache.v_core[:, :, :m].cpu()
     kt, vt = to_bits(cache.k_tail), to_bits(cache.v_tail)
@@ -104,3 +108,4 @@ def test_decode_64k_256_steps(cca):
         steps = np.arange(wl.steps) if b == 0 else sampled
         O_ref = oracle.attend_rows(qf, kf, vf, Kc_ref, Vc_ref, wl.g, wl.w, rows_all[steps])
         assert_close(O[b:b + 1, :, steps].numpy(), O_ref, None, f"decode b={b}")
+        assert_close(O16[b:b + 1, :, steps], O_ref, None, f"decode bf16 b={b}")
