@@ -4,7 +4,7 @@ One step is one pass of the whole hot path over synthetic inputs:
   prefill  cca_pool + cca_attn_prefill on a LLaMA2-7B-shaped layer at 128K
            context (B=1, H=32, d=128, T=131072, g=16, w=1024; bf16 N(0,1)
            inputs, 1% of key rows x4);
-  decode   256 x (cca_cache_append + cca_attn_decode) with B=8, H=32,
+  decode   256 x cca_decode_step (append + attention, one launch) with B=8, H=32,
            d=128, g=16, w=1024 against a cache built from a 65536-token
            prefix (4096 core slots + a 1040-token raw ring).
 value = prefill tokens/s (whole job, all ranks); decode latency per token
@@ -48,6 +48,15 @@ UNIT = "tokens/s"
 PREFILL = synth.PREFILL_128K
 DECODE = synth.DECODE_64K
 L2_BYTES = 126 * 2 ** 20
+# the other prefill workloads of the method's evaluation shapes, timed beside
+# the headline one
+EXTRA_PREFILL = (synth.PREFILL_32K.name, synth.GQA_16K.name)
+TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.md")
+# the sources of the prefill kernel: DRAM counters taken on another version
+# of them do not describe this one
+PREFILL_SOURCES = ("long_context_sparse_cca_b200/csrc/prefill.cu",
+                   "long_context_sparse_cca_b200/csrc/sm100.cuh",
+                   "long_context_sparse_cca_b200/csrc/common.cuh")
 
 
 # ----------------------------------------------------------------- workload arithmetic
@@ -72,6 +81,32 @@ def pool_bytes(wl) -> float:
     m = wl.T // wl.g
     return 2.0 * (2 * wl.B * wl.Hkv * wl.T * wl.d + wl.B * wl.Hq * m * wl.d +
                   2 * wl.B * wl.Hkv * m * wl.d)
+
+
+def prefill_bytes(wl) -> float:
+    """Algorithmic DRAM bytes of the fused attention: Q, K, V and the core
+    keys/values read once, O written once (2-byte elements)."""
+    m = wl.T // wl.g
+    return 2.0 * (2 * wl.B * wl.Hq * wl.T * wl.d + 2 * wl.B * wl.Hkv * wl.T * wl.d +
+                  2 * wl.B * wl.Hkv * m * wl.d)
+
+
+def prefill_entry(wl, t: dict, pk: dict, world: int) -> dict:
+    """Tokens/s and roofline fractions of one prefill workload from its
+    pool and prefill times (ms)."""
+    flops = prefill_flops(wl)
+    tf = flops / (t["prefill_ms"] * 1e-3) / 1e12
+    gbs = pool_bytes(wl) / (t["pool_ms"] * 1e-3) / 1e9
+    out = {"tokens_per_s": world * wl.B * wl.T / ((t["pool_ms"] + t["prefill_ms"]) * 1e-3),
+           "pool_ms": t["pool_ms"], "prefill_ms": t["prefill_ms"],
+           "prefill_tflops": tf, "algorithmic_flops": flops,
+           "prefill_frac_burst": tf / pk["bf16_tflops"],
+           "prefill_frac_sustained": (tf / pk["bf16_tflops_sustained"]
+                                      if pk["bf16_tflops_sustained"] else None),
+           "pool_gbs": gbs, "pool_frac": gbs / pk["hbm_gbs"],
+           "traffic": measured_traffic(wl.name),
+           "algorithmic_bytes": prefill_bytes(wl)}
+    return out
 
 
 def decode_bytes(wl, t: int) -> float:
@@ -109,6 +144,32 @@ def peaks() -> dict:
                 "source": "measured"}
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0,
             "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def prefill_source_hash() -> str:
+    import hashlib
+    h = hashlib.sha256()
+    for rel in PREFILL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_traffic(workload: str):
+    """DRAM bytes (read + write) of one prefill-kernel launch on `workload`,
+    from the committed ncu summary, or None when that summary is missing,
+    names another workload, or was taken on other kernel sources.  The
+    summary holds machine-readable lines `traffic <workload> <bytes>
+    <source hash>`."""
+    if not os.path.exists(TRAFFIC_PROFILE):
+        return None
+    want = prefill_source_hash()
+    with open(TRAFFIC_PROFILE) as f:
+        for line in f:
+            parts = line.strip().strip("`").split()
+            if len(parts) == 4 and parts[0] == "traffic" and parts[1] == workload:
+                return float(parts[2]) if parts[3] == want else None
+    return None
 
 
 # ----------------------------------------------------------------- clocks
@@ -253,7 +314,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         del y
         o_t = torch.empty((dw.B, dw.Hq, dw.d), dtype=torch.bfloat16, device="cuda")
         ws_bytes = cca.cca_decode_workspace_bytes(cache)
-        workspace = torch.empty(ws_bytes, dtype=torch.uint8, device="cuda")
+        # zero-filled once, as cca_decode_step requires of a new workspace
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device="cuda")
     st = cca.cca_device_status()
     assert st == cca.CCA_OK, cca.status_string(st)
 
@@ -272,8 +334,8 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         cache.len = dw.T  # same 256 steps every time (slots rewritten identically)
         evs[0].record(stream)
         for s in range(dw.steps):
-            cca.cca_cache_append(cache, new_q[s], new_k[s], new_v[s])
-            cca.cca_attn_decode(cache, new_q[s], o_t, workspace=workspace)
+            # append + decode attention of the token, one launch
+            cca.cca_decode_step(cache, new_q[s], new_k[s], new_v[s], o_t, workspace=workspace)
         evs[1].record(stream)
 
     def step(ev_p, ev_d):
@@ -327,17 +389,60 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         if i > 0:  # first one warms the pinned paths
             e2e_ms.append(a.elapsed_time(b))
 
+    # --- the other prefill workloads, each timed on its own after the
+    # headline step (kernels entries, not the bench value)
+    extra = {}
+    for name in ([] if args.no_extra else EXTRA_PREFILL):
+        if not do_prefill:
+            break
+        extra[name] = time_prefill(cca, synth.WORKLOADS[name], args.steps, args.warmup,
+                                   stream, torch)
+
     # one all-reduce of every timing, the same on all ranks (no e2e: -1)
     total_ms, mean_pool, mean_prefill, mean_decode, mean_e2e = max_over_ranks(
         [total_ms, float(np.mean(pool_ms)), float(np.mean(prefill_ms)),
          float(np.mean(decode_ms)), float(np.mean(e2e_ms)) if e2e_ms else -1.0],
         world, "cuda")
     mean_e2e = mean_e2e if mean_e2e >= 0 else None
+    for name in list(extra):
+        extra[name] = dict(zip(("pool_ms", "prefill_ms"),
+                               max_over_ranks([extra[name]["pool_ms"],
+                                               extra[name]["prefill_ms"]], world, "cuda")))
     h2d = 3 * Q.numel() * 2 if do_prefill else 0
     d2h = O.numel() * 2 if do_prefill else 0
     return dict(total_ms=total_ms, pool_ms=mean_pool, prefill_ms=mean_prefill,
                 decode_ms=mean_decode, e2e_ms=mean_e2e, clocks=clk.summary(),
-                h2d=h2d, d2h=d2h)
+                h2d=h2d, d2h=d2h, extra=extra)
+
+
+def time_prefill(cca, wl, steps: int, warmup: int, stream, torch) -> dict:
+    """Mean CUDA-event times (ms) of cca_pool and cca_attn_prefill on one
+    prefill workload, inputs resident in HBM, after `warmup` untimed
+    passes; the buffers are freed afterwards."""
+    x = synth.generate(wl)
+    Q, K, V = _dev(x.q, torch), _dev(x.k, torch), _dev(x.v, torch)
+    del x
+    m = wl.T // wl.g
+    Kc = torch.empty((wl.B, wl.Hkv, m, wl.d), dtype=torch.float16, device="cuda")
+    Vc = torch.empty_like(Kc)
+    O = torch.empty((wl.B, wl.Hq, wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(warmup + steps)]
+    for e in evs:
+        e[0].record(stream)
+        cca.cca_pool(Q, K, V, wl.g, Kc, Vc)
+        e[1].record(stream)
+        cca.cca_attn_prefill(Q, K, V, Kc, Vc, wl.g, wl.w, O=O)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    st = cca.cca_device_status()
+    assert st == cca.CCA_OK, cca.status_string(st)
+    timed = evs[warmup:]
+    out = {"pool_ms": float(np.mean([e[0].elapsed_time(e[1]) for e in timed])),
+           "prefill_ms": float(np.mean([e[1].elapsed_time(e[2]) for e in timed]))}
+    del Q, K, V, Kc, Vc, O
+    torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------- oracle (CPU) arm
@@ -438,6 +543,18 @@ def oracle_single_thread_value(budget_s: float = 3.0) -> float:
 
 # ----------------------------------------------------------------- main
 
+def config_dict(args, world: int) -> dict:
+    """The workload description both arms print (the same keys and values,
+    so the two lines describe one configuration)."""
+    pw = args.prefill_wl
+    return {"workload": pw.name, "decode_workload": DECODE.name,
+            "parts": args.parts,
+            "global_batch": pw.B * world, "seq_len": pw.T,
+            "parallelism": f"replicas{world}", "core_dtype": "f16",
+            "o_dtype": "bf16",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
 def main(argv=None) -> int:
     ap = argparse.ArgumentParser(description=__doc__,
                                  formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -453,6 +570,8 @@ def main(argv=None) -> int:
                     choices=[w.name for w in synth.WORKLOADS.values() if w.steps == 0],
                     help="prefill workload (profiling runs; the default is the headline)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip timing the 32K and GQA prefill workloads")
     args = ap.parse_args(argv)
     args.prefill_wl = synth.WORKLOADS[args.prefill_workload]
     if args.warmup < 3:
@@ -480,8 +599,7 @@ def main(argv=None) -> int:
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": sec * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
                 "dtype": "f64", "data": "synthetic", "impl": "reference",
-                "config": {"workload": PREFILL.name, "seq_len": PREFILL.T,
-                           "global_batch": PREFILL.B},
+                "config": config_dict(args, world),
                 "cpu_baseline": cb,
                 "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
@@ -513,25 +631,22 @@ def main(argv=None) -> int:
                             for t in range(DECODE.T, DECODE.T + DECODE.steps)]))
     dec_gbs = dbytes / (nz(dec_us) * 1e-6) / 1e9
     pool_gbs = pbytes / (nz(r["pool_ms"]) * 1e-3) / 1e9
-    launches = args.steps * ((2 if do_prefill else 0) + (2 * DECODE.steps if do_decode else 0))
+    launches = args.steps * ((2 if do_prefill else 0) + (DECODE.steps if do_decode else 0))
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": r["total_ms"] / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": pw.name, "decode_workload": DECODE.name,
-                   "parts": args.parts,
-                   "global_batch": pw.B * world, "seq_len": pw.T,
-                   "parallelism": f"replicas{world}", "core_dtype": "f16",
-                   "o_dtype": "bf16",
-                   "l2": "inputs larger than L2 (no flush)"},
+        "config": config_dict(args, world),
         "decode_us_per_step": dec_us,
         "roofline": {"bound": "tensor", "kernel": "cca_attn_prefill",
                      "achieved": achieved_tf, "peak": pk["bf16_tflops"],
                      "unit": "TFLOP/s", "frac": achieved_tf / pk["bf16_tflops"],
-                     "traffic": None, "peak_source": pk["source"] + " (burst)",
-                     "algorithmic_flops": flops},
+                     "traffic": measured_traffic(pw.name),
+                     "peak_source": pk["source"] + " (burst)",
+                     "algorithmic_flops": flops,
+                     "algorithmic_bytes": prefill_bytes(pw)},
         "kernels": {
             "cca_attn_prefill": {"ms": r["prefill_ms"], "tflops": achieved_tf,
                                  "frac_burst": achieved_tf / pk["bf16_tflops"],
@@ -541,7 +656,9 @@ def main(argv=None) -> int:
                          "frac": pool_gbs / pk["hbm_gbs"], "bytes": pbytes},
             "decode_step": {"us": dec_us, "gbs": dec_gbs, "frac": dec_gbs / pk["hbm_gbs"],
                             "bytes": dbytes,
-                            "launches": "cca_cache_append + cca_attn_decode (ticket memset + split kernel with fused merge)"},
+                            "launches": "cca_decode_step: one kernel per token (append, split-K attention, merge)"},
+            **{f"prefill[{name}]": prefill_entry(synth.WORKLOADS[name], t, pk, world)
+               for name, t in r["extra"].items()},
         },
         "kv_cache": cache_bytes(pw, pw.T),
         "clocks": r["clocks"],

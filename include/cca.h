@@ -127,9 +127,13 @@ cca_status cca_attn_prefill(const void *Q, const void *K, const void *V,
                             cudaStream_t stream);
 
 /*
- * Fill a cache from a prefix of T tokens (Q, K, V as for cca_pool): pools
- * every complete group into its core slot and copies the last
- * min(T, tail_cap) raw tokens into their ring slots; sets c->len = T.
+ * Fill a cache from a prefix of T tokens (Q, K, V as for cca_pool).  The
+ * write-up's section 基于 Triton 的底层加速 gives the operator KV-cache
+ * support for prefill and decode; section 计算和存储效率对比 measures the
+ * cache's size against full attention.  This call pools every complete
+ * group into its core slot (section 全局感知池化) and copies the last
+ * min(T, tail_cap) raw tokens into their ring slots (the window of
+ * section 局部保留模块); it sets c->len = T.
  * CCA_ERR_CAPACITY if floor((T - 1) / g) >= core_cap.  The cache's shape
  * fields (B, Hq, Hkv, d, g, w, core_cap, tail_cap) must be set.
  */
@@ -137,11 +141,12 @@ cca_status cca_cache_prefill(cca_cache *c, const void *Q, const void *K,
                              const void *V, int64_t T, cudaStream_t stream);
 
 /*
- * Append one token t = c->len per batch row: q_t [B, Hq, d], k_t, v_t
- * [B, Hkv, d] (bf16).  k_t, v_t go to ring slot t % tail_cap; if the token
- * completes group j = t / g ((t + 1) % g == 0), that group is pooled from
- * the ring with the token's own queries (it is the group's last token) into
- * core slot j.  On success c->len becomes t + 1.  CCA_ERR_CAPACITY (nothing
+ * Append one token t = c->len per batch row (KV-cache support, section
+ * 基于 Triton 的底层加速; pooling of a completed group, section
+ * 全局感知池化): q_t [B, Hq, d], k_t, v_t [B, Hkv, d] (bf16).  k_t, v_t
+ * go to ring slot t % tail_cap; if the token completes group j = t / g
+ * ((t + 1) % g == 0), that group is pooled from the ring with the token's
+ * own queries (it is the group's last token) into core slot j.  On success c->len becomes t + 1.  CCA_ERR_CAPACITY (nothing
  * written) if t / g >= core_cap.
  */
 cca_status cca_cache_append(cca_cache *c, const void *q_t, const void *k_t,
@@ -153,7 +158,9 @@ size_t cca_decode_workspace_bytes(const cca_cache *c);
 
 /*
  * Attention of the newest token t = c->len - 1 over the cache: core slots
- * j < ws(t)/g and ring slots of tokens ws(t)..t, one softmax.
+ * j < ws(t)/g and ring slots of tokens ws(t)..t, one softmax (the fused
+ * core + local attention of sections 局部保留模块 and 全局-局部模块可微融合,
+ * for one query, from the cache of section 基于 Triton 的底层加速).
  *   q_t [B, Hq, d] (bf16), o_t [B, Hq, d] written in o_dtype.
  * Split over key ranges; partial results go to `workspace` (device memory
  * of at least cca_decode_workspace_bytes(c) bytes, 256-byte aligned, its
@@ -166,12 +173,43 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                            size_t workspace_bytes, cudaStream_t stream);
 
 /*
- * Per-row lengths in device memory.  These two calls read each batch row's
- * length from `lens` (device memory, B entries of long long, 8-byte
+ * One decode step in one launch: cca_cache_append of token t = c->len
+ * followed by cca_attn_decode of that token, fused into a single kernel
+ * (the write-up's section 基于 Triton 的底层加速 describes one
+ * cache-friendly operator with native KV-cache support; sections
+ * 全局感知池化, 局部保留模块 and 全局-局部模块可微融合 define what it
+ * computes).  Arguments as for the two calls: q_t [B, Hq, d], k_t, v_t
+ * [B, Hkv, d] (bf16), o_t [B, Hq, d] in o_dtype.  The results, and the
+ * cache contents afterwards, equal those of the two separate calls.  On
+ * success c->len becomes t + 1; CCA_ERR_CAPACITY (nothing launched) if
+ * t / g >= core_cap.
+ * Workspace: as for cca_attn_decode (cca_decode_workspace_bytes(c) bytes,
+ * 256-byte aligned), but this call does not clear the completion counters
+ * it keeps there: zero-fill a workspace once before its first use with a
+ * cache (e.g. cudaMemsetAsync(ws, 0, bytes, stream)).  Every decode call of
+ * this library (this one, cca_attn_decode, cca_attn_decode_rows) leaves the
+ * counters at zero when it completes, so the workspace stays ready for the
+ * next call on the same cache.  Calls sharing a workspace must not overlap
+ * on the GPU.
+ */
+cca_status cca_decode_step(cca_cache *c, const void *q_t, const void *k_t, const void *v_t,
+                           void *o_t, cca_dtype o_dtype, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Per-row lengths in device memory (the same cache append and decode
+ * attention as above, sections 基于 Triton 的底层加速, 全局感知池化,
+ * 局部保留模块 and 全局-局部模块可微融合).  These two calls read each batch
+ * row's length from `lens` (device memory, B entries of long long, 8-byte
  * aligned) instead of c->len, so rows may have different lengths and a
  * sequence of decode steps can be captured once in a CUDA graph and
  * replayed (nothing the host must know changes from step to step).
- * c->len is neither read nor written.
+ * c->len is neither read nor written.  lens[b] must be the number of tokens
+ * row b holds: as set when the row was filled (cca_cache_prefill of that
+ * row) and advanced by cca_cache_append_rows.  The library cannot tell a
+ * larger value from a real length: a row whose lens[b] runs ahead of what
+ * was appended is decoded from stale ring and core slots, and only a length
+ * beyond the cache's capacity is reported.
  *
  * cca_cache_append_rows: row b appends its token t = lens[b] exactly as
  * cca_cache_append does (ring slot t % tail_cap, pooling of group t / g when
@@ -185,8 +223,9 @@ cca_status cca_cache_append_rows(const cca_cache *c, long long *lens, const void
                                  const void *k_t, const void *v_t, cudaStream_t stream);
 
 /*
- * cca_attn_decode_rows: cca_attn_decode for token t_b = lens[b] - 1 of
- * every row b, each over its own core slots and ring window.  The workspace
+ * cca_attn_decode_rows (sections 局部保留模块 and 全局-局部模块可微融合 for
+ * one query per row): cca_attn_decode for token t_b = lens[b] - 1 of every
+ * row b, each over its own core slots and ring window.  The workspace
  * is the same as cca_attn_decode's.  A row with lens[b] == 0 gets a zero
  * output; a row longer than the cache gets a zero output and
  * cca_device_status() reports CCA_ERR_CAPACITY.
@@ -211,8 +250,10 @@ cca_status cca_attn_decode_rows(const cca_cache *c, const long long *lens, const
  * on until the process exits; it allocates nothing.
  *   Returns CCA_ERR_SCRATCH (nothing launched) if the cache needs more
  *   workspace than that array; other errors as cca_attn_decode.
- *   The first call on a device looks up the array's device address (with
- *   that device current), so make it before any stream capture begins.
+ *   The first call in each CUDA context (once per device for the runtime's
+ *   primary contexts, and again after a context is re-created, e.g. after
+ *   cudaDeviceReset) looks up the array's device address with that context
+ *   current, so make it before any stream capture begins.
  *   All calls share the array: calls whose kernels may overlap on the GPU
  *   (e.g. on unordered streams) race.  Nothing in it needs clearing.
  */

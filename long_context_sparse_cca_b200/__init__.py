@@ -10,7 +10,8 @@ Build the library with ``python -m long_context_sparse_cca_b200.build``.
 
 Entry points (same names as the C ABI):
     cca_pool, cca_attn_prefill, cca_cache_prefill, cca_cache_append,
-    cca_attn_decode, cca_decode_workspace_bytes, cca_attn_decode_noalloc,
+    cca_attn_decode, cca_decode_step (append + decode in one launch),
+    cca_decode_workspace_bytes, cca_attn_decode_noalloc,
     cca_cache_append_rows, cca_attn_decode_rows (per-row lengths in device
     memory), cca_selftest_wait_timeout, cca_device_status
 and the ``Cache`` class holding a decode cache's device buffers.
@@ -42,7 +43,7 @@ EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
            "cca_device_status", "cca_status_string", "cca_version", "cca_last_error",
            "cca_attn_decode_noalloc", "cca_selftest_wait_timeout",
-           "cca_cache_append_rows", "cca_attn_decode_rows")
+           "cca_cache_append_rows", "cca_attn_decode_rows", "cca_decode_step")
 
 
 class CCAError(RuntimeError):
@@ -91,6 +92,8 @@ def lib():
     L.cca_attn_decode.restype = st
     L.cca_attn_decode_noalloc.argtypes = [CP, P, P, i, P]
     L.cca_attn_decode_noalloc.restype = st
+    L.cca_decode_step.argtypes = [CP, P, P, P, P, i, P, ctypes.c_size_t, P]
+    L.cca_decode_step.restype = st
     L.cca_cache_append_rows.argtypes = [CP, P, P, P, P, P]
     L.cca_cache_append_rows.restype = st
     L.cca_attn_decode_rows.argtypes = [CP, P, P, P, i, P, ctypes.c_size_t, P]
@@ -312,16 +315,42 @@ def cca_attn_decode(cache: Cache, q_t, o_t=None, out_dtype=None,
         dt = torch.bfloat16 if out_dtype is None else out_dtype
         o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
     od = _odtype(o_t.dtype)
-    nbytes = cca_decode_workspace_bytes(cache)
     if workspace is None:
-        if cache.workspace is None or cache.workspace.numel() < nbytes:
-            cache.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8,
-                                          device=q_t.device)
-        workspace = cache.workspace
+        workspace = _cache_workspace(cache, q_t.device)
     _check(lib().cca_attn_decode(
         ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(o_t, "o_t", o_t.dtype),
         od, ctypes.c_void_p(workspace.data_ptr()), workspace.numel(),
         _stream(stream)), "cca_attn_decode")
+    return o_t
+
+
+def _cache_workspace(cache: Cache, device):
+    """The cache's own decode workspace, zero-filled when (re)allocated, as
+    cca_decode_step requires before its first use."""
+    torch = _torch()
+    nbytes = cca_decode_workspace_bytes(cache)
+    if cache.workspace is None or cache.workspace.numel() < nbytes:
+        cache.workspace = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
+    return cache.workspace
+
+
+def cca_decode_step(cache: Cache, q_t, k_t, v_t, o_t=None, out_dtype=None,
+                    workspace=None, stream=None):
+    """Append token t = cache.len and return its attention output, in one
+    launch: q_t [B,Hq,d], k_t/v_t [B,Hkv,d] (bf16) -> o_t [B,Hq,d].  A
+    caller-provided workspace must have been zero-filled before its first
+    use with this cache."""
+    torch = _torch()
+    if o_t is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
+    od = _odtype(o_t.dtype)
+    if workspace is None:
+        workspace = _cache_workspace(cache, q_t.device)
+    _check(lib().cca_decode_step(
+        ctypes.byref(cache.struct), _dev(q_t, "q_t"), _dev(k_t, "k_t"), _dev(v_t, "v_t"),
+        _dev(o_t, "o_t", o_t.dtype), od, ctypes.c_void_p(workspace.data_ptr()),
+        workspace.numel(), _stream(stream)), "cca_decode_step")
     return o_t
 
 
@@ -354,12 +383,8 @@ def cca_attn_decode_rows(cache: Cache, lens, q_t, o_t=None, out_dtype=None,
         dt = torch.bfloat16 if out_dtype is None else out_dtype
         o_t = torch.empty(tuple(q_t.shape), dtype=dt, device=q_t.device)
     od = _odtype(o_t.dtype)
-    nbytes = cca_decode_workspace_bytes(cache)
     if workspace is None:
-        if cache.workspace is None or cache.workspace.numel() < nbytes:
-            cache.workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8,
-                                          device=q_t.device)
-        workspace = cache.workspace
+        workspace = _cache_workspace(cache, q_t.device)
     _check(lib().cca_attn_decode_rows(
         ctypes.byref(cache.struct), _lens(lens), _dev(q_t, "q_t"),
         _dev(o_t, "o_t", o_t.dtype), od, ctypes.c_void_p(workspace.data_ptr()),

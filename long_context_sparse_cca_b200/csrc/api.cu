@@ -185,6 +185,34 @@ cca_status cca_attn_decode(const cca_cache *c, const void *q_t, void *o_t,
                                         c->tail_cap, t, stream));
 }
 
+cca_status cca_decode_step(cca_cache *c, const void *q_t, const void *k_t, const void *v_t,
+                           void *o_t, cca_dtype o_dtype, void *workspace,
+                           size_t workspace_bytes, cudaStream_t stream)
+{
+    const cca_status s = cache_status(c);
+    if (s != CCA_OK) return s;
+    if (o_dtype != CCA_BF16 && o_dtype != CCA_F32) return CCA_ERR_INVALID_ARG;
+    if (!ptr_ok(q_t, true) || !ptr_ok(k_t, true) || !ptr_ok(v_t, true) || !ptr_ok(o_t, true) ||
+        workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+        return CCA_ERR_INVALID_ARG;
+    if (workspace_bytes < cca::decode_workspace_bytes(c->B, c->Hq, c->Hkv, c->d, c->core_cap,
+                                                      c->tail_cap))
+        return CCA_ERR_INVALID_ARG;
+    const int64_t t = c->len;
+    if (t >= kMaxT || t / c->g >= c->core_cap) return CCA_ERR_CAPACITY;
+    const size_t out = size_t(c->B) * c->Hq * c->d * (o_dtype == CCA_F32 ? 4 : 2);
+    const size_t in_q = size_t(c->B) * c->Hq * c->d * 2, in_kv = size_t(c->B) * c->Hkv * c->d * 2;
+    if (overlap(o_t, out, q_t, in_q) || overlap(o_t, out, k_t, in_kv) ||
+        overlap(o_t, out, v_t, in_kv) || overlap(o_t, out, workspace, workspace_bytes))
+        return CCA_ERR_INVALID_ARG;
+    const cudaError_t e = cca::launch_decode_step(
+        c->k_core, c->v_core, c->k_tail, c->v_tail, q_t, k_t, v_t, o_t, o_dtype == CCA_F32,
+        workspace, c->B, c->Hq, c->Hkv, c->d, c->g, c->w, c->core_cap, c->tail_cap, t, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    c->len = t + 1;
+    return CCA_OK;
+}
+
 cca_status cca_cache_append_rows(const cca_cache *c, long long *lens, const void *q_t,
                                  const void *k_t, const void *v_t, cudaStream_t stream)
 {

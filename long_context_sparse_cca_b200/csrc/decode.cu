@@ -14,6 +14,8 @@
 #include "common.cuh"
 #include "internal.h"
 
+#include <algorithm>
+
 namespace cca {
 
 __device__ unsigned int g_decode_status;  // kStatusCapacity
@@ -58,19 +60,156 @@ __device__ __forceinline__ void row8_to_f32(const uint4 v, bool core, float (&f)
 struct CacheView {
     const uint16_t *k_core, *v_core, *k_tail, *v_tail;
     int64_t core_cap, tail_cap, ws, n_core;
+    int64_t ws_slot;  // ws % tail_cap: ring slot of the window's first token
     // Row of key k (0 <= k < n_keys) of pair bh: core slot k, or the ring
-    // slot of raw token ws + (k - n_core).
+    // slot of raw token ws + (k - n_core).  The window holds at most
+    // tail_cap tokens, so one wrap-around step replaces a modulo.
     __device__ __forceinline__ int64_t row(int64_t bh, int64_t k, bool &core) const
     {
         core = k < n_core;
-        return core ? bh * core_cap + k
-                    : bh * tail_cap + (ws + (k - n_core)) % tail_cap;
+        if (core) return bh * core_cap + k;
+        int64_t slot = ws_slot + (k - n_core);
+        if (slot >= tail_cap) slot -= tail_cap;
+        return bh * tail_cap + slot;
     }
 };
 
+// The token a fused decode step appends (cca_decode_step).  Its key/value
+// rows are read from these inputs, not from the ring slot this launch
+// writes; the CTA with a pair's last split writes that ring slot and, when
+// the token completes a group, pools the group into its core slot.  No key
+// any CTA of the launch reads is written by it: the ring slot of token t
+// held token t - tail_cap, before the window, and core slot t / g is not in
+// token t's core set.
+struct StepArgs {
+    const uint16_t *k_t, *v_t;                    // [B, Hkv, D] rows of token t
+    uint16_t *k_core, *v_core, *k_tail, *v_tail;  // the cache, written
+    int g;
+    int64_t t;
+};
+
+// The append of a fused step for pair bh, by the whole CTA with the
+// decode kernel's own lane layout (lane kl of a row slot kg holds 16 bytes
+// of a row), so that the kernel's register budget does not grow: the ring
+// slot of token t, and when t completes group j = t / g, the pooling of
+// that group (section 全局感知池化: the scores of the group's keys against
+// the queries of its last token, token t, soft-maxed per query head and
+// averaged over the r heads, weight the group's keys and values; the same
+// arithmetic as the separate append: fp32 scores, exp2f, fp32 sums, fp16
+// rows).  Scratch: lg (r g + g floats) and red (NG D floats).
 template <int D, int R>
+__device__ __forceinline__ void step_append(const StepArgs &st, const uint16_t *q_t,
+                                            int64_t b, int64_t h, int Hq,
+                                            int64_t bh, int r, int64_t tail_cap,
+                                            int64_t core_cap, float scale_log2, float *lg,
+                                            float *red)
+{
+    using S = DecodeShape<D>;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kl = lane % S::KL, kg = warp * S::KPW + lane / S::KL;
+    const int64_t slot = bh * tail_cap + st.t % tail_cap;
+    for (int c = tid; c < D / 8; c += kDecodeThreads) {
+        reinterpret_cast<uint4 *>(st.k_tail + slot * D)[c] =
+            reinterpret_cast<const uint4 *>(st.k_t + bh * D)[c];
+        reinterpret_cast<uint4 *>(st.v_tail + slot * D)[c] =
+            reinterpret_cast<const uint4 *>(st.v_t + bh * D)[c];
+    }
+    const int g = st.g;
+    if ((st.t + 1) % g != 0) return;
+    const int64_t j = st.t / g;
+    const int first_slot = static_cast<int>((st.t - g + 1) % tail_cap);
+    const int cap = static_cast<int>(tail_cap);
+    // row i of the group: the ring slot of token t - g + 1 + i (g <= tail_cap:
+    // one wrap-around step), or for the last one (token t) the input row
+    auto grow = [&](const uint16_t *ring, const uint16_t *in, int i) {
+        int slot = first_slot + i;
+        if (slot >= cap) slot -= cap;
+        return i == g - 1 ? in + bh * D : ring + (bh * tail_cap + slot) * D;
+    };
+    float *logit = lg, *weight = lg + r * g;
+    // the scoring queries: token t's own (it is the group's last token)
+    float q[R][8];
+#pragma unroll
+    for (int k = 0; k < R; ++k)
+        if (k < r)
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(q_t + (b * Hq + h * r + k) * D + kl * 8),
+                          q[k]);
+    // scores (loop bound uniform per warp: the shuffles need every lane)
+    for (int base = 0; base < g; base += S::NG) {
+        const int i = base + kg;
+        float kf[8];
+        if (i < g)
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(grow(st.k_tail, st.k_t, i) + kl * 8), kf);
+        else
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kf[e] = 0.f;
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            if (k < r) {
+                float sc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sc = fmaf(q[k][e], kf[e], sc);
+#pragma unroll
+                for (int o = 1; o < S::KL; o <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+                if (kl == 0 && i < g) logit[k * g + i] = sc * scale_log2;
+            }
+        }
+    }
+    __syncthreads();
+    // per query head: softmax over the g scores (numerators left in logit)
+    for (int k = warp; k < r; k += kDecodeThreads / 32) {
+        float mx = -INFINITY;
+        for (int i = lane; i < g; i += 32) mx = fmaxf(mx, logit[k * g + i]);
+        mx = warp_max(mx);
+        float sum = 0.f;
+        for (int i = lane; i < g; i += 32) {
+            const float e = exp2f(logit[k * g + i] - mx);
+            logit[k * g + i] = e;
+            sum += e;
+        }
+        sum = warp_sum(sum);
+        if (lane == 0) red[k] = (1.0f / static_cast<float>(r)) / sum;
+    }
+    __syncthreads();
+    for (int i = tid; i < g; i += kDecodeThreads) {
+        float wi = 0.f;
+        for (int k = 0; k < r; ++k) wi += logit[k * g + i] * red[k];
+        weight[i] = wi;
+    }
+    __syncthreads();
+    // pooled key, then pooled value: per-slot partial sums, then a sum over
+    // the row slots through shared memory
+    bool over = false;
+    for (int which = 0; which < 2; ++which) {
+        const uint16_t *ring = which ? st.v_tail : st.k_tail;
+        const uint16_t *in = which ? st.v_t : st.k_t;
+        float acc[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+        for (int i = kg; i < g; i += S::NG) {
+            float f[8];
+            bf16x8_to_f32(*reinterpret_cast<const uint4 *>(grow(ring, in, i) + kl * 8), f);
+            const float wi = weight[i];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] = fmaf(wi, f[e], acc[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[kg * D + kl * 8 + e] = acc[e];
+        __syncthreads();
+        uint16_t *out = (which ? st.v_core : st.k_core) + (bh * core_cap + j) * D;
+        for (int c = tid; c < D; c += kDecodeThreads) {
+            float sum = 0.f;
+            for (int s = 0; s < S::NG; ++s) sum += red[s * D + c];
+            out[c] = __half_as_ushort(__float2half_rn(clamp_f16(sum, over)));
+        }
+        __syncthreads();
+    }
+    if (__syncthreads_or(over) && tid == 0) atomicOr(&g_decode_status, kStatusRange);
+}
+
+template <int D, int R, bool STEP>
 __global__ void __launch_bounds__(kDecodeThreads)
-    decode_split_kernel(CacheView cv, const uint16_t *__restrict__ q_t,
+    decode_split_kernel(CacheView cv, StepArgs st, const uint16_t *__restrict__ q_t,
                         float *__restrict__ part_o, float2 *__restrict__ part_ml,
                         unsigned int *__restrict__ tickets, void *__restrict__ o_t,
                         int out_f32, int Hq, int Hkv, int64_t n_keys, int chunk,
@@ -80,8 +219,10 @@ __global__ void __launch_bounds__(kDecodeThreads)
     using S = DecodeShape<D>;
     extern __shared__ float dsm[];
     const int r = Hq / Hkv;
-    float *lg = dsm;                               // [R][chunk]
-    float *red = dsm + R * chunk;                  // [NG][R][D]
+    // [R][chunk] scores (a fused step's pooling also uses it: (r + 1) g)
+    const int lg_floats = STEP ? max(R * chunk, (r + 1) * st.g) : R * chunk;
+    float *lg = dsm;
+    float *red = dsm + lg_floats;                  // [NG][R][D]
     float *stat = red + S::NG * R * D;             // [R][2]
     const int split = blockIdx.x;
     const int64_t bh = blockIdx.y;
@@ -110,6 +251,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             return;
         }
         cvb.ws = wsb;
+        cvb.ws_slot = wsb % cv.tail_cap;
         cvb.n_core = wsb / g;
         n_keys = cvb.n_core + (tb - wsb + 1);
         nsplit = static_cast<int>((n_keys + chunk - 1) / chunk);
@@ -131,10 +273,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
     }
 
+    // The keys streamed from the cache: all of the chunk, except (fused
+    // step, last split) the appended token, whose rows come from the inputs
+    // and are added after each loop, outside the hot path.
+    const bool new_key = STEP && split == nsplit - 1;
+    const int nkc = new_key ? nk - 1 : nk;
+
     // Scores of this chunk's keys, all query heads at once.  The loop bound
     // is the same for every lane (the shuffles below need the whole warp);
     // each lane's key i = base + kg + u * NG is guarded instead.
-    for (int base = 0; base < nk; base += 4 * S::NG) {
+    for (int base = 0; base < nkc; base += 4 * S::NG) {
         const int i0 = base + kg;
         uint4 kv[4];
         bool kcore[4];
@@ -143,7 +291,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const int i = i0 + u * S::NG;
             kv[u] = make_uint4(0u, 0u, 0u, 0u);
             kcore[u] = false;
-            if (i < nk) {
+            if (i < nkc) {
                 const int64_t row = cvb.row(bh, c0 + i, kcore[u]);
                 const uint16_t *src = kcore[u] ? cv.k_core : cv.k_tail;
                 kv[u] = ldg_stream(src + row * D + kl * 8);
@@ -163,8 +311,24 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
                     for (int o = 1; o < S::KL; o <<= 1)
                         s += __shfl_xor_sync(0xffffffffu, s, o);
-                    if (kl == 0 && i < nk) lg[k * chunk + i] = s * scale_log2;
+                    if (kl == 0 && i < nkc) lg[k * chunk + i] = s * scale_log2;
                 }
+            }
+        }
+    }
+    if (new_key && warp == 0) {
+        // the appended token's scores (the upper half-warp repeats them)
+        float kf[8];
+        bf16x8_to_f32(ldg_stream(st.k_t + bh * D + kl * 8), kf);
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            if (k < r) {
+                float sc = 0.f;
+#pragma unroll
+                for (int e = 0; e < 8; ++e) sc = fmaf(q[k][e], kf[e], sc);
+#pragma unroll
+                for (int o = 1; o < S::KL; o <<= 1) sc += __shfl_xor_sync(0xffffffffu, sc, o);
+                if (lane == 0) lg[k * chunk + nk - 1] = sc * scale_log2;
             }
         }
     }
@@ -195,7 +359,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
     for (int k = 0; k < R; ++k)
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[k][e] = 0.f;
-    for (int base = 0; base < nk; base += 4 * S::NG) {
+    for (int base = 0; base < nkc; base += 4 * S::NG) {
         const int i0 = base + kg;
         uint4 vv[4];
         bool vcore[4];
@@ -204,7 +368,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
             const int i = i0 + u * S::NG;
             vv[u] = make_uint4(0u, 0u, 0u, 0u);
             vcore[u] = false;
-            if (i < nk) {
+            if (i < nkc) {
                 const int64_t row = cvb.row(bh, c0 + i, vcore[u]);
                 const uint16_t *src = vcore[u] ? cv.v_core : cv.v_tail;
                 vv[u] = ldg_stream(src + row * D + kl * 8);
@@ -213,7 +377,7 @@ __global__ void __launch_bounds__(kDecodeThreads)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
             const int i = i0 + u * S::NG;
-            if (i < nk) {
+            if (i < nkc) {
                 float vf[8];
                 row8_to_f32(vv[u], vcore[u], vf);
 #pragma unroll
@@ -224,6 +388,19 @@ __global__ void __launch_bounds__(kDecodeThreads)
                         for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(p, vf[e], acc[k][e]);
                     }
                 }
+            }
+        }
+    }
+    if (new_key && kg == 0) {
+        // the appended token's value row, into row slot 0's sums
+        float vf[8];
+        bf16x8_to_f32(ldg_stream(st.v_t + bh * D + kl * 8), vf);
+#pragma unroll
+        for (int k = 0; k < R; ++k) {
+            if (k < r) {
+                const float p = lg[k * chunk + nk - 1];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) acc[k][e] = fmaf(p, vf[e], acc[k][e]);
             }
         }
     }
@@ -243,6 +420,16 @@ __global__ void __launch_bounds__(kDecodeThreads)
         if (c == 0) part_ml[qrow] = make_float2(stat[2 * k], stat[2 * k + 1]);
     }
 
+    if (STEP && split == nsplit - 1) {
+        // the append (ring slot of token t, pooling of the group it
+        // completes), after this CTA's own keys, so that none of its state
+        // is live in the loops above; nothing this launch reads is written
+        // here.  Scratch: the score and partial-sum buffers, free now (the
+        // merge below uses them again only after the barrier).
+        __syncthreads();
+        step_append<D, R>(st, q_t, b, h, Hq, bh, r, cv.tail_cap, cv.core_cap, scale_log2, lg,
+                          red);
+    }
     // Ticket: the CTA that takes the last one merges.  The fence makes this
     // CTA's partials visible device-wide before its ticket is counted.
     __threadfence();
@@ -321,24 +508,32 @@ __global__ void __launch_bounds__(kDecodeThreads)
         }
         __syncthreads();
     }
+    // Every CTA of this pair has taken its ticket: leave the counter at zero
+    // for the next call (a fused step relies on it; the other calls also
+    // clear it first).
+    if (tid == 0) tickets[bh] = 0u;
 }
 
-template <int D, int R>
+template <int D, int R, bool STEP = false>
 cudaError_t launch_split(const CacheView &cv, const void *q_t, float *part_o,
                          float2 *part_ml, unsigned int *tickets, void *o_t, bool o_f32,
                          int B, int Hq, int Hkv, int64_t n_keys, int nsplit,
                          float scale_log2, cudaStream_t s, const long long *lens = nullptr,
-                         int g = 0, int w = 0, int64_t core_cap = 0, int stride = 0)
+                         int g = 0, int w = 0, int64_t core_cap = 0, int stride = 0,
+                         const StepArgs &st = StepArgs{})
 {
     using S = DecodeShape<D>;
-    const size_t smem =
-        sizeof(float) * (R * kDecodeChunk + S::NG * R * D + 2 * R);
-    auto kern = decode_split_kernel<D, R>;
+    // score buffer (a fused step pools a group in it: (r + 1) g floats),
+    // partial sums, statistics; the same layout as the kernel's
+    const int r = Hq / Hkv;
+    const int lg_floats = STEP ? std::max(R * kDecodeChunk, (r + 1) * st.g) : R * kDecodeChunk;
+    const size_t smem = sizeof(float) * (lg_floats + S::NG * R * D + 2 * R);
+    auto kern = decode_split_kernel<D, R, STEP>;
     if (smem > 48 * 1024)
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem));
     dim3 grid(nsplit, B * Hkv);
-    kern<<<grid, kDecodeThreads, smem, s>>>(cv, static_cast<const uint16_t *>(q_t),
+    kern<<<grid, kDecodeThreads, smem, s>>>(cv, st, static_cast<const uint16_t *>(q_t),
                                             part_o, part_ml, tickets, o_t, o_f32 ? 1 : 0,
                                             Hq, Hkv, n_keys, kDecodeChunk, nsplit,
                                             scale_log2, lens, g, w, core_cap, stride);
@@ -409,7 +604,8 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
                  core_cap,
                  tail_cap,
                  p.ws,
-                 p.n_core};
+                 p.n_core,
+                 p.ws % tail_cap};
     const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
     const int r = Hq / Hkv;
     // the tickets start at zero on every call (the workspace is not
@@ -419,6 +615,61 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
 #define CCA_SPLIT(DD, RR)                                                          \
     e = launch_split<DD, RR>(cv, q_t, part_o, part_ml, tickets, o_t, o_f32, B, Hq, \
                              Hkv, p.n_keys, p.nsplit, scale_log2, s)
+    if (d == 128) {
+        if (r == 1) CCA_SPLIT(128, 1);
+        else if (r == 2) CCA_SPLIT(128, 2);
+        else if (r <= 4) CCA_SPLIT(128, 4);
+        else if (r <= 8) CCA_SPLIT(128, 8);
+        else CCA_SPLIT(128, 16);
+    } else {
+        if (r == 1) CCA_SPLIT(64, 1);
+        else if (r == 2) CCA_SPLIT(64, 2);
+        else if (r <= 4) CCA_SPLIT(64, 4);
+        else if (r <= 8) CCA_SPLIT(64, 8);
+        else CCA_SPLIT(64, 16);
+    }
+#undef CCA_SPLIT
+    return e;
+}
+
+cudaError_t launch_decode_step(void *k_core, void *v_core, void *k_tail, void *v_tail,
+                               const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               bool o_f32, void *workspace, int B, int Hq, int Hkv, int d,
+                               int g, int w, int64_t core_cap, int64_t tail_cap, int64_t t,
+                               cudaStream_t s)
+{
+    const DecodePlan p = decode_plan(t, g, w, B, Hkv);
+    const WorkspaceLayout L = workspace_layout(B, Hq, Hkv, d, core_cap, tail_cap);
+    char *ws = static_cast<char *>(workspace);
+    float *part_o = reinterpret_cast<float *>(ws);
+    float2 *part_ml = reinterpret_cast<float2 *>(ws + L.o_bytes);
+    unsigned int *tickets = reinterpret_cast<unsigned int *>(ws + L.o_bytes + L.ml_bytes);
+    CacheView cv{static_cast<const uint16_t *>(k_core),
+                 static_cast<const uint16_t *>(v_core),
+                 static_cast<const uint16_t *>(k_tail),
+                 static_cast<const uint16_t *>(v_tail),
+                 core_cap,
+                 tail_cap,
+                 p.ws,
+                 p.n_core,
+                 p.ws % tail_cap};
+    StepArgs st{static_cast<const uint16_t *>(k_t),
+                static_cast<const uint16_t *>(v_t),
+                static_cast<uint16_t *>(k_core),
+                static_cast<uint16_t *>(v_core),
+                static_cast<uint16_t *>(k_tail),
+                static_cast<uint16_t *>(v_tail),
+                g,
+                t};
+    const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));
+    const int r = Hq / Hkv;
+    // no ticket clearing here: every call leaves the tickets at zero, and a
+    // new workspace is zero-filled by its owner (see cca_decode_step)
+    cudaError_t e = cudaSuccess;
+#define CCA_SPLIT(DD, RR)                                                                \
+    e = launch_split<DD, RR, true>(cv, q_t, part_o, part_ml, tickets, o_t, o_f32, B, Hq,  \
+                                   Hkv, p.n_keys, p.nsplit, scale_log2, s, nullptr, 0, 0, \
+                                   0, 0, st)
     if (d == 128) {
         if (r == 1) CCA_SPLIT(128, 1);
         else if (r == 2) CCA_SPLIT(128, 2);
@@ -456,6 +707,7 @@ cudaError_t launch_decode_rows(const void *k_core, const void *v_core,
                  static_cast<const uint16_t *>(v_tail),
                  core_cap,
                  tail_cap,
+                 0,
                  0,
                  0};
     const float scale_log2 = kLog2e / sqrtf(static_cast<float>(d));

@@ -48,6 +48,16 @@ cudaError_t launch_decode(const void *k_core, const void *v_core,
                           int g, int w, int64_t core_cap, int64_t tail_cap,
                           int64_t t, cudaStream_t s);
 
+// One decode step in one launch: append token t (k_t, v_t; ring slot, and
+// pooling of the group it completes) and the attention of token t.  The
+// workspace's tickets must be zero on entry (every decode launch leaves them
+// so).
+cudaError_t launch_decode_step(void *k_core, void *v_core, void *k_tail, void *v_tail,
+                               const void *q_t, const void *k_t, const void *v_t, void *o_t,
+                               bool o_f32, void *workspace, int B, int Hq, int Hkv, int d,
+                               int g, int w, int64_t core_cap, int64_t tail_cap, int64_t t,
+                               cudaStream_t s);
+
 // Fused core + local attention over a whole sequence (tcgen05 kernel).
 cudaError_t launch_prefill(const void *Q, const void *K, const void *V,
                            const void *Kc, const void *Vc, void *O, bool o_f32,

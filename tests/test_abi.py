@@ -118,6 +118,33 @@ def test_cache_checks(L):
                              ws, None) == cca.CCA_ERR_INVALID_ARG  # dtype
 
 
+def test_decode_step_argument_checks(L):
+    """cca_decode_step refuses bad arguments and a full cache before any
+    launch, and leaves the cache length unchanged."""
+    P = ctypes.c_void_p
+    c = _cache(length=10)
+    ws = L.cca_decode_workspace_bytes(ctypes.byref(c))
+    args = lambda q=FAKE, k=FAKE + 8192, v=FAKE + 16384, o=FAKE + 4096, dt=0, w=FAKE, n=ws: (  # noqa: E731
+        ctypes.byref(c), P(q), P(k), P(v), P(o), dt, P(w), n, None)
+    assert L.cca_decode_step(*args(q=0)) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_decode_step(*args(k=FAKE + 8)) == cca.CCA_ERR_INVALID_ARG  # misaligned
+    assert L.cca_decode_step(*args(n=ws - 1)) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_decode_step(*args(w=FAKE + 16)) == cca.CCA_ERR_INVALID_ARG  # 256-byte
+    assert L.cca_decode_step(*args(dt=3)) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_decode_step(*args(o=FAKE)) == cca.CCA_ERR_INVALID_ARG  # o_t overlaps q_t
+    assert c.len == 10
+    c = _cache(core_cap=2, length=32)  # token 32 belongs to group 2: no slot
+    ws = L.cca_decode_workspace_bytes(ctypes.byref(c))
+    assert L.cca_decode_step(ctypes.byref(c), P(FAKE), P(FAKE + 8192), P(FAKE + 16384),
+                             P(FAKE + 4096), 0, P(FAKE + (8 << 20)), ws,
+                             None) == cca.CCA_ERR_CAPACITY
+    assert c.len == 32
+    bad = _cache(tail_cap=10)
+    assert L.cca_decode_step(ctypes.byref(bad), P(FAKE), P(FAKE + 8192), P(FAKE + 16384),
+                             P(FAKE + 4096), 0, P(FAKE), 1 << 20,
+                             None) == cca.CCA_ERR_INVALID_ARG
+
+
 def test_noalloc_decode_refuses_oversized_cache(L):
     """A cache whose decode workspace exceeds the library's fixed scratch is
     refused before anything touches the GPU."""
