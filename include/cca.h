@@ -127,6 +127,50 @@ cca_status cca_attn_prefill(const void *Q, const void *K, const void *V,
                             cudaStream_t stream);
 
 /*
+ * Training: the forward attention of cca_attn_prefill that also writes
+ * each row's log-sum-exp, lse [B, Hq, T] (fp32, device memory, log2 units:
+ * lse[t] = log2 of the sum over t's keys of 2^(q_t . key * log2(e) /
+ * sqrt(d))), which cca_attn_backward reads.  Other arguments, results and
+ * errors as cca_attn_prefill.
+ */
+cca_status cca_attn_prefill_lse(const void *Q, const void *K, const void *V, const void *Kc,
+                                const void *Vc, void *O, cca_dtype o_dtype, float *lse, int B,
+                                int Hq, int Hkv, int64_t T, int d, int g, int w,
+                                cudaStream_t stream);
+
+/* Bytes of device workspace cca_attn_backward needs for these shapes
+ * (0 for an invalid shape). */
+size_t cca_attn_backward_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int g);
+
+/*
+ * Backward pass for training (the write-up's section 全局-局部模块可微融合
+ * calls the global-local fusion differentiable, and its section 基于 Triton
+ * 的底层加速 says the fused operator serves training): for an upstream
+ * gradient dO of the attention output, the gradients of
+ * L = sum(dO * O) with respect to Q, K and V, through the fused attention
+ * (queries, raw window keys/values, pooled core keys/values) and through
+ * the pooling (section 全局感知池化: each group's weights come from its last
+ * query and its keys).
+ *   Q, K, V, Kc, Vc as for cca_attn_prefill; O and lse from
+ *   cca_attn_prefill_lse on the same inputs (O in o_dtype); dO [B, Hq, T, d]
+ *   bf16.  dQ [B, Hq, T, d], dK, dV [B, Hkv, T, d]: fp32, written.
+ *   workspace: cca_attn_backward_workspace_bytes bytes of device memory,
+ *   256-byte aligned (fp16 copies of Q and dO, per-row sums, fp32 core
+ *   gradients; the call clears what it accumulates).  r = Hq / Hkv <= 32.
+ * Runs as four launches on `stream` (per-row sums; dQ on tcgen05 tensor
+ * cores, one query tile per CTA; dK, dV on tcgen05, one key tile per CTA;
+ * the pooling's chain rule, one warp per group).  Errors as
+ * cca_attn_prefill; values beyond the fp16 range in Q or dO are clamped in
+ * the core stream's copies and reported as CCA_ERR_RANGE.
+ */
+cca_status cca_attn_backward(const void *Q, const void *K, const void *V, const void *Kc,
+                             const void *Vc, const void *O, cca_dtype o_dtype,
+                             const float *lse, const void *dO, float *dQ, float *dK,
+                             float *dV, int B, int Hq, int Hkv, int64_t T, int d, int g,
+                             int w, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream);
+
+/*
  * Fill a cache from a prefix of T tokens (Q, K, V as for cca_pool).  The
  * write-up's section 基于 Triton 的底层加速 gives the operator KV-cache
  * support for prefill and decode; section 计算和存储效率对比 measures the

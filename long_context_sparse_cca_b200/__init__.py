@@ -10,6 +10,8 @@ Build the library with ``python -m long_context_sparse_cca_b200.build``.
 
 Entry points (same names as the C ABI):
     cca_pool, cca_attn_prefill, cca_cache_prefill, cca_cache_append,
+    cca_attn_prefill_lse (forward that keeps each row's log-sum-exp),
+    cca_attn_backward, cca_attn_backward_workspace_bytes (training),
     cca_attn_decode, cca_decode_step (append + decode in one launch),
     cca_decode_workspace_bytes, cca_attn_decode_noalloc,
     cca_cache_append_rows, cca_attn_decode_rows (per-row lengths in device
@@ -43,7 +45,8 @@ EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_cache_append", "cca_decode_workspace_bytes", "cca_attn_decode",
            "cca_device_status", "cca_status_string", "cca_version", "cca_last_error",
            "cca_attn_decode_noalloc", "cca_selftest_wait_timeout",
-           "cca_cache_append_rows", "cca_attn_decode_rows", "cca_decode_step")
+           "cca_cache_append_rows", "cca_attn_decode_rows", "cca_decode_step",
+           "cca_attn_prefill_lse", "cca_attn_backward", "cca_attn_backward_workspace_bytes")
 
 
 class CCAError(RuntimeError):
@@ -82,6 +85,13 @@ def lib():
     L.cca_pool.restype = st
     L.cca_attn_prefill.argtypes = [P, P, P, P, P, P, i, i, i, i, i64, i, i, i, P]
     L.cca_attn_prefill.restype = st
+    L.cca_attn_prefill_lse.argtypes = [P, P, P, P, P, P, i, P, i, i, i, i64, i, i, i, P]
+    L.cca_attn_prefill_lse.restype = st
+    L.cca_attn_backward_workspace_bytes.argtypes = [i, i, i, i64, i, i]
+    L.cca_attn_backward_workspace_bytes.restype = ctypes.c_size_t
+    L.cca_attn_backward.argtypes = [P, P, P, P, P, P, i, P, P, P, P, P, i, i, i, i64, i, i, i,
+                                    P, ctypes.c_size_t, P]
+    L.cca_attn_backward.restype = st
     L.cca_cache_prefill.argtypes = [CP, P, P, P, i64, P]
     L.cca_cache_prefill.restype = st
     L.cca_cache_append.argtypes = [CP, P, P, P, P]
@@ -213,6 +223,59 @@ def cca_attn_prefill(Q, K, V, Kc, Vc, g: int, w: int, O=None,
         _dev(Vc, "Vc", torch.float16), _dev(O, "O", O.dtype), od, B, Hq, Hkv, T, d, int(g),
         int(w), _stream(stream)), "cca_attn_prefill")
     return O
+
+
+def cca_attn_prefill_lse(Q, K, V, Kc, Vc, g: int, w: int, O=None, out_dtype=None,
+                         lse=None, stream=None):
+    """cca_attn_prefill that also returns each row's log-sum-exp (fp32
+    [B, Hq, T], log2 units), as cca_attn_backward needs: (O, lse)."""
+    torch = _torch()
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    if O is None:
+        dt = torch.bfloat16 if out_dtype is None else out_dtype
+        O = torch.empty((B, Hq, T, d), dtype=dt, device=Q.device)
+    if lse is None:
+        lse = torch.empty((B, Hq, T), dtype=torch.float32, device=Q.device)
+    od = _odtype(O.dtype)
+    if tuple(O.shape) != (B, Hq, T, d) or tuple(lse.shape) != (B, Hq, T):
+        raise ValueError("O must be [B, Hq, T, d] and lse [B, Hq, T]")
+    _check(lib().cca_attn_prefill_lse(
+        _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(Kc, "Kc", torch.float16),
+        _dev(Vc, "Vc", torch.float16), _dev(O, "O", O.dtype), od,
+        _dev(lse, "lse", torch.float32), B, Hq, Hkv, T, d, int(g), int(w), _stream(stream)),
+        "cca_attn_prefill_lse")
+    return O, lse
+
+
+def cca_attn_backward_workspace_bytes(B: int, Hq: int, Hkv: int, T: int, d: int, g: int) -> int:
+    return int(lib().cca_attn_backward_workspace_bytes(int(B), int(Hq), int(Hkv), int(T),
+                                                       int(d), int(g)))
+
+
+def cca_attn_backward(Q, K, V, Kc, Vc, O, lse, dO, g: int, w: int, dQ=None, dK=None,
+                      dV=None, workspace=None, stream=None):
+    """Gradients (dQ, dK, dV), fp32, of sum(dO * O) for the CCA attention
+    O = attention(Q, K, V) with its pooled Kc, Vc (from cca_pool) and the
+    forward's O and lse (from cca_attn_prefill_lse).  dO: bf16 like Q."""
+    torch = _torch()
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    f32 = dict(dtype=torch.float32, device=Q.device)
+    dQ = torch.empty((B, Hq, T, d), **f32) if dQ is None else dQ
+    dK = torch.empty((B, Hkv, T, d), **f32) if dK is None else dK
+    dV = torch.empty((B, Hkv, T, d), **f32) if dV is None else dV
+    nbytes = cca_attn_backward_workspace_bytes(B, Hq, Hkv, T, d, g)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=Q.device)
+    _check(lib().cca_attn_backward(
+        _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), _dev(Kc, "Kc", torch.float16),
+        _dev(Vc, "Vc", torch.float16), _dev(O, "O", O.dtype), _odtype(O.dtype),
+        _dev(lse, "lse", torch.float32), _dev(dO, "dO"), _dev(dQ, "dQ", torch.float32),
+        _dev(dK, "dK", torch.float32), _dev(dV, "dV", torch.float32), B, Hq, Hkv, T, d, int(g),
+        int(w), ctypes.c_void_p(workspace.data_ptr()), workspace.numel(), _stream(stream)),
+        "cca_attn_backward")
+    return dQ, dK, dV
 
 
 class Cache:

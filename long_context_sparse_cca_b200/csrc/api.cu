@@ -115,6 +115,83 @@ cca_status cca_attn_prefill(const void *Q, const void *K, const void *V, const v
                                          Hkv, T, d, g, w, stream));
 }
 
+cca_status cca_attn_prefill_lse(const void *Q, const void *K, const void *V, const void *Kc,
+                                const void *Vc, void *O, cca_dtype o_dtype, float *lse, int B,
+                                int Hq, int Hkv, int64_t T, int d, int g, int w,
+                                cudaStream_t stream)
+{
+    const cca_status s = shape_status(B, Hq, Hkv, T, d, g, w);
+    if (s != CCA_OK) return s;
+    if (o_dtype != CCA_BF16 && o_dtype != CCA_F32) return CCA_ERR_INVALID_ARG;
+    const bool any = T > 0;
+    const int64_t m = T / g;
+    if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(O, any) ||
+        !ptr_ok(lse, any) || !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
+        return CCA_ERR_INVALID_ARG;
+    if (!any) return CCA_OK;
+    const int64_t n_items = ((T + 255) / 256) * int64_t(B) * Hq;
+    if (n_items > INT32_MAX) return CCA_ERR_UNSUPPORTED;
+    const size_t esz = o_dtype == CCA_F32 ? 4 : 2;
+    const size_t out = size_t(B) * Hq * T * d * esz, lse_b = size_t(B) * Hq * T * 4;
+    const size_t in_q = size_t(B) * Hq * T * d * 2, in_kv = size_t(B) * Hkv * T * d * 2;
+    const size_t in_c = size_t(B) * Hkv * m * d * 2;
+    if (overlap(O, out, Q, in_q) || overlap(O, out, K, in_kv) || overlap(O, out, V, in_kv) ||
+        overlap(O, out, Kc, in_c) || overlap(O, out, Vc, in_c) || overlap(lse, lse_b, O, out) ||
+        overlap(lse, lse_b, Q, in_q) || overlap(lse, lse_b, K, in_kv) ||
+        overlap(lse, lse_b, V, in_kv) || overlap(lse, lse_b, Kc, in_c) ||
+        overlap(lse, lse_b, Vc, in_c))
+        return CCA_ERR_INVALID_ARG;
+    return from_cuda(cca::launch_prefill(Q, K, V, Kc, Vc, O, o_dtype == CCA_F32, B, Hq, Hkv, T,
+                                         d, g, w, stream, lse));
+}
+
+size_t cca_attn_backward_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int d, int g)
+{
+    if (shape_status(B, Hq, Hkv, T, d, g, 0) != CCA_OK) return 0;
+    return cca::bw_layout(B, Hq, Hkv, T, d, g).total;
+}
+
+cca_status cca_attn_backward(const void *Q, const void *K, const void *V, const void *Kc,
+                             const void *Vc, const void *O, cca_dtype o_dtype,
+                             const float *lse, const void *dO, float *dQ, float *dK,
+                             float *dV, int B, int Hq, int Hkv, int64_t T, int d, int g,
+                             int w, void *workspace, size_t workspace_bytes,
+                             cudaStream_t stream)
+{
+    const cca_status s = shape_status(B, Hq, Hkv, T, d, g, w);
+    if (s != CCA_OK) return s;
+    if (o_dtype != CCA_BF16 && o_dtype != CCA_F32) return CCA_ERR_INVALID_ARG;
+    if (Hq / Hkv > 32) return CCA_ERR_UNSUPPORTED;
+    const bool any = T > 0;
+    const int64_t m = T / g;
+    if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(O, any) ||
+        !ptr_ok(lse, any) || !ptr_ok(dO, any) || !ptr_ok(dQ, any) || !ptr_ok(dK, any) ||
+        !ptr_ok(dV, any) || !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
+        return CCA_ERR_INVALID_ARG;
+    if (!any) return CCA_OK;
+    if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||
+        workspace_bytes < cca::bw_layout(B, Hq, Hkv, T, d, g).total)
+        return CCA_ERR_INVALID_ARG;
+    if (((T + 127) / 128) * int64_t(B) * Hq > INT32_MAX) return CCA_ERR_UNSUPPORTED;
+    // the outputs alias nothing the call reads, nor each other, nor the workspace
+    const size_t nq = size_t(B) * Hq * T * d, nk = size_t(B) * Hkv * T * d;
+    const size_t nc = size_t(B) * Hkv * m * d;
+    const void *ins[9] = {Q, K, V, Kc, Vc, O, lse, dO, workspace};
+    const size_t in_n[9] = {nq * 2, nk * 2, nk * 2, nc * 2, nc * 2,
+                            nq * (o_dtype == CCA_F32 ? 4 : 2), size_t(B) * Hq * T * 4, nq * 2,
+                            workspace_bytes};
+    void *outs[3] = {dQ, dK, dV};
+    const size_t out_n[3] = {nq * 4, nk * 4, nk * 4};
+    for (int i = 0; i < 3; ++i) {
+        for (int j = 0; j < 9; ++j)
+            if (overlap(outs[i], out_n[i], ins[j], in_n[j])) return CCA_ERR_INVALID_ARG;
+        for (int j = i + 1; j < 3; ++j)
+            if (overlap(outs[i], out_n[i], outs[j], out_n[j])) return CCA_ERR_INVALID_ARG;
+    }
+    return from_cuda(cca::launch_backward(Q, K, V, Kc, Vc, O, o_dtype == CCA_F32, lse, dO, dQ, dK,
+                                          dV, B, Hq, Hkv, T, d, g, w, workspace, stream));
+}
+
 cca_status cca_cache_prefill(cca_cache *c, const void *Q, const void *K, const void *V,
                              int64_t T, cudaStream_t stream)
 {
@@ -253,14 +330,15 @@ cca_status cca_device_status(cudaStream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int a = 0, b = 0, c = 0, d = 0, f = 0;
+    unsigned int a = 0, b = 0, c = 0, d = 0, f = 0, h = 0;
     if ((e = cca::prefill_status_read_clear(&a)) != cudaSuccess ||
         (e = cca::pool_status_read_clear(&b)) != cudaSuccess ||
         (e = cca::append_status_read_clear(&c)) != cudaSuccess ||
         (e = cca::selftest_status_read_clear(&d)) != cudaSuccess ||
-        (e = cca::decode_status_read_clear(&f)) != cudaSuccess)
+        (e = cca::decode_status_read_clear(&f)) != cudaSuccess ||
+        (e = cca::backward_status_read_clear(&h)) != cudaSuccess)
         return from_cuda(e);
-    const unsigned int st = a | b | c | d | f;
+    const unsigned int st = a | b | c | d | f | h;
     if (st & cca::kStatusTimeout) return CCA_ERR_TIMEOUT;
     if (st & cca::kStatusCapacity) return CCA_ERR_CAPACITY;
     if (st & cca::kStatusRange) return CCA_ERR_RANGE;

@@ -1,0 +1,1046 @@
+// cca_attn_backward: gradients of CCA attention for training.
+//
+// The write-up calls the global-local fusion differentiable (section
+// 全局-局部模块可微融合) and its fused operator serves training (section 基于
+// Triton 的底层加速).  For upstream gradients dO of the fused attention output
+// O, this computes dQ, dK, dV of L = sum(dO * O), where O depends on Q, K, V
+// directly (queries; raw keys/values of the local window) and through the
+// pooled core keys/values (section 全局感知池化).  With logits
+// x = (q . key) / sqrt(d), P = softmax(x) per row (from the forward's
+// log-sum-exp), dP = dO . value and D = rowsum(dO * O):
+//   dS = P (dP - D),  dQ = sum dS key / sqrt(d),
+//   dKey = sum dS q / sqrt(d),  dValue = sum P dO,
+// for raw keys (dK, dV) and core keys (dKc, dVc); then the pooling's chain
+// rule moves dKc, dVc onto the group's keys, values and scoring queries.
+//
+// Launches, in order on the caller's stream:
+//   1. bw_prep_kernel: D = rowsum(dO * O); fp16 copies of Q and dO for the
+//      core stream (core keys/values are fp16, and an MMA takes one type);
+//   2. bw_dq_kernel (tcgen05): per 128-row query tile, over its key tiles
+//      (local then core): S = Q K^T, dP = dO V^T, dS, dQ += dS K;
+//   3. bw_dkv_kernel (tcgen05): per 128-key tile, over the query tiles and
+//      query heads that see it: S^T = K Q^T, dP^T = V dO^T, dV += P^T dO,
+//      dK += dS^T Q; raw tiles store dK, dV; core tiles (whose query range
+//      is long, so it is cut into chunks) add into fp32 dKc, dVc;
+//   4. bw_pool_kernel: one warp per group, the pooling's chain rule.
+#include "common.cuh"
+#include "internal.h"
+#include "sm100.cuh"
+#include "tma_map.h"
+
+namespace cca {
+
+__device__ unsigned int g_backward_status;  // kStatusTimeout | kStatusRange
+
+namespace {
+
+constexpr uint64_t kBwWaitNs = 2000000000ull;  // 2 s per wait
+constexpr int kCoreChunk = 16;                 // query tiles per core work item
+
+template <int D>
+struct Bt {
+    static constexpr int NBOX = D / 64;
+    static constexpr int BOX_BYTES = 128 * 128;
+    static constexpr int TILE_BYTES = BOX_BYTES * NBOX;  // 128 rows x D, 16-bit
+};
+
+struct BwParams {
+    int B, Hq, Hkv, r, T, g, w, m;
+    float scale;       // 1 / sqrt(d)
+    float scale_log2;  // log2(e) / sqrt(d)
+    const float *lse;  // [B, Hq, T], log2 units
+    const float *Dv;   // [B, Hq, T]
+    float *dQ;         // [B, Hq, T, d]
+    float *dK, *dV;    // [B, Hkv, T, d]
+    float *dKc, *dVc;  // [B, Hkv, m, d], accumulated (zero on entry)
+    int n_qt, n_kt, n_ct;
+    int n_items, n_core_items;
+};
+
+__device__ __forceinline__ int ws_of(int t, int g, int w)
+{
+    const int lo = t > w ? t - w : 0;
+    return (lo / g) * g;
+}
+
+// Shared helpers of the two tcgen05 kernels ---------------------------------
+
+struct BwBars {
+    uint64_t q_full[2], q_empty[2];  // query-side tiles (Q, dO)
+    uint64_t k_full[4], k_empty[4];  // key-side ring (dQ kernel)
+    uint64_t v_full[4], v_empty[4];
+    uint64_t kv_full, kv_empty;      // key-side tiles (dK/dV kernel)
+    uint64_t s_full, s_free, p_full, mm_done, acc_empty, drain;
+    uint32_t tmem_base;
+    int abort, never;
+};
+
+__device__ __forceinline__ void bw_timeout(BwBars *bars)
+{
+    atomicOr(&g_backward_status, kStatusTimeout);
+    *reinterpret_cast<volatile int *>(&bars->abort) = 1;
+}
+
+__device__ __forceinline__ bool bw_lane_wait(uint64_t *bar, uint32_t parity, BwBars *bars)
+{
+    const bool ok = wait_bounded(bar, parity, &bars->abort, kBwWaitNs);
+    if (!ok) bw_timeout(bars);
+    return ok;
+}
+
+__device__ __forceinline__ bool bw_warp_wait(uint64_t *bar, uint32_t parity, BwBars *bars)
+{
+    bool ok = wait_bounded(bar, parity, &bars->abort, kBwWaitNs);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok && (threadIdx.x & 31) == 0) bw_timeout(bars);
+    return ok;
+}
+
+// 128 x 128 x D product into TMEM columns, both operands K-major in shared
+// memory (128-byte swizzled TMA tiles).
+template <int D>
+__device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint32_t idesc)
+{
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        constexpr uint32_t box16 = Bt<D>::BOX_BYTES >> 4;
+        const uint32_t off = (kk >> 2) * box16 + (kk & 3) * 2;
+        mma_ss(d_tmem, a0 + off, b0 + off, idesc, kk > 0 ? 1u : 0u);
+    }
+}
+
+// 128 x D x 128 product: A (16-bit pairs) in TMEM, B MN-major in shared
+// memory; accumulate unless `first`.
+__device__ __forceinline__ void mma_tm(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                       uint32_t idesc, bool first)
+{
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc, (first && kk == 0) ? 0u : 1u);
+}
+
+__device__ __forceinline__ uint32_t pack16(float a, float b, bool f16)
+{
+    return f16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
+}
+
+// 1. D = rowsum(dO * O) and the fp16 copies --------------------------------
+
+template <int D, bool OF32>
+__global__ void bw_prep_kernel(const uint16_t *__restrict__ dO, const void *__restrict__ O,
+                               const uint16_t *__restrict__ Q, float *__restrict__ Dv,
+                               uint16_t *__restrict__ Q16, uint16_t *__restrict__ dO16,
+                               int64_t rows)
+{
+    const int lane = threadIdx.x & 31;
+    constexpr int DPL = D / 32;
+    bool over = false;
+    for (int64_t row = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+         row < rows; row += (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5) {
+        const int64_t base = row * D + lane * DPL;
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < DPL; e += 2) {
+            const uint32_t g2 = *reinterpret_cast<const uint32_t *>(dO + base + e);
+            const uint32_t q2 = *reinterpret_cast<const uint32_t *>(Q + base + e);
+            float o0, o1;
+            if (OF32) {
+                const float2 o = *reinterpret_cast<const float2 *>(
+                    static_cast<const float *>(O) + base + e);
+                o0 = o.x;
+                o1 = o.y;
+            } else {
+                const uint32_t o2 =
+                    *reinterpret_cast<const uint32_t *>(static_cast<const uint16_t *>(O) + base + e);
+                o0 = bf16_lo(o2);
+                o1 = bf16_hi(o2);
+            }
+            s = fmaf(bf16_lo(g2), o0, s);
+            s = fmaf(bf16_hi(g2), o1, s);
+            *reinterpret_cast<uint32_t *>(dO16 + base + e) =
+                pack_f16x2(clamp_f16(bf16_lo(g2), over), clamp_f16(bf16_hi(g2), over));
+            *reinterpret_cast<uint32_t *>(Q16 + base + e) =
+                pack_f16x2(clamp_f16(bf16_lo(q2), over), clamp_f16(bf16_hi(q2), over));
+        }
+        s = warp_sum(s);
+        if (lane == 0) Dv[row] = s;
+    }
+    if (__any_sync(0xffffffffu, over) && lane == 0) atomicOr(&g_backward_status, kStatusRange);
+}
+
+// 2. dQ ---------------------------------------------------------------------
+//
+// Work item: one 128-row query tile of one (batch, query head), latest tiles
+// first.  Key tiles as in the forward: local (raw keys ws(t0) .. last row,
+// bf16) then core (pooled keys 0 .. ws(last)/g - 1, fp16, against the fp16
+// copies of Q and dO, reloaded at the switch).  Warps 0-3: one query row per
+// thread; warp 4: TMA producer; warp 5: MMA issuer (one thread).
+// TMEM: S [0,128), dP [128,256), dS [256,320) (16-bit pairs), dQ [320, +D).
+template <int D>
+struct BqLayout {
+    using T = Bt<D>;
+    static constexpr int KST = D == 128 ? 3 : 4, VST = D == 128 ? 2 : 4;
+    static constexpr int OFF_Q = 0, OFF_DO = T::TILE_BYTES;
+    static constexpr int OFF_K = 2 * T::TILE_BYTES;
+    static constexpr int OFF_V = OFF_K + KST * T::TILE_BYTES;
+    static constexpr int OFF_BAR = OFF_V + VST * T::TILE_BYTES;
+    static constexpr int SMEM = OFF_BAR + 512 + 1024;
+    static constexpr uint32_t S_COL = 0, DP_COL = 128, DS_COL = 256, DQ_COL = 320;
+};
+
+struct QGeom {
+    int b, hq, h, t0, tlast, ws_lo, n_local, n_core, n_tiles;
+};
+
+__device__ __forceinline__ QGeom q_geom(int item, const BwParams &p)
+{
+    QGeom G;
+    const int bhq = p.B * p.Hq;
+    const int qt = p.n_qt - 1 - item / bhq;
+    const int x = item - (item / bhq) * bhq;
+    G.b = x / p.Hq;
+    G.hq = x - G.b * p.Hq;
+    G.h = G.hq / p.r;
+    G.t0 = qt * 128;
+    G.tlast = min(G.t0 + 127, p.T - 1);
+    G.ws_lo = ws_of(G.t0, p.g, p.w);
+    G.n_local = (G.tlast - G.ws_lo + 1 + 127) / 128;
+    G.n_core = (ws_of(G.tlast, p.g, p.w) / p.g + 127) / 128;
+    G.n_tiles = G.n_local + G.n_core;
+    return G;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bw_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                 const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
+                 const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                 const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                 const BwParams p)
+{
+    using L = BqLayout<D>;
+    using T = Bt<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sQ = smem + L::OFF_Q, *sO = smem + L::OFF_DO;
+    uint8_t *sK = smem + L::OFF_K, *sV = smem + L::OFF_V;
+    BwBars *bars = reinterpret_cast<BwBars *>(smem + L::OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int bhq = p.B * p.Hq;
+    const int n_items = p.n_qt * bhq;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&bars->q_full[0], 1);
+        mbar_init(&bars->q_empty[0], 1);
+        for (int s = 0; s < L::KST; ++s) {
+            mbar_init(&bars->k_full[s], 1);
+            mbar_init(&bars->k_empty[s], 1);
+        }
+        for (int s = 0; s < L::VST; ++s) {
+            mbar_init(&bars->v_full[s], 1);
+            mbar_init(&bars->v_empty[s], 1);
+        }
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->s_free, 4);
+        mbar_init(&bars->p_full, 4);
+        mbar_init(&bars->mm_done, 1);
+        mbar_init(&bars->acc_empty, 4);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        bars->never = 0;
+        mbar_fence_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t kc = 0, vc = 0, qc = 0;
+            bool ok = true;
+            auto load_q = [&](const CUtensorMap *mq, const CUtensorMap *mo, const QGeom &G) {
+                if (qc > 0 && !(ok = bw_lane_wait(&bars->q_empty[0], (qc - 1) & 1, bars)))
+                    return;
+                mbar_arrive_expect_tx(&bars->q_full[0], 2 * T::TILE_BYTES);
+                const int z = G.b * p.Hq + G.hq;
+                for (int bx = 0; bx < T::NBOX; ++bx) {
+                    tma_load_3d(sQ + bx * T::BOX_BYTES, mq, &bars->q_full[0], bx * 64, G.t0, z);
+                    tma_load_3d(sO + bx * T::BOX_BYTES, mo, &bars->q_full[0], bx * 64, G.t0, z);
+                }
+                ++qc;
+            };
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const QGeom G = q_geom(item, p);
+                load_q(&tmQ, &tmO, G);
+                const int z = G.b * p.Hkv + G.h;
+                for (int j = 0; ok && j < G.n_tiles; ++j) {
+                    const bool core = j >= G.n_local;
+                    if (core && j == G.n_local) {
+                        load_q(&tmQ16, &tmO16, G);
+                        if (!ok) break;
+                    }
+                    const int key0 = core ? (j - G.n_local) * 128 : G.ws_lo + j * 128;
+                    const int s = kc % L::KST;
+                    if (!(ok = bw_lane_wait(&bars->k_empty[s], ((kc / L::KST) & 1) ^ 1, bars))) break;
+                    mbar_arrive_expect_tx(&bars->k_full[s], T::TILE_BYTES);
+                    for (int bx = 0; bx < T::NBOX; ++bx)
+                        tma_load_3d(sK + s * T::TILE_BYTES + bx * T::BOX_BYTES, core ? &tmKc : &tmK,
+                                    &bars->k_full[s], bx * 64, key0, z);
+                    ++kc;
+                    const int sv = vc % L::VST;
+                    if (!(ok = bw_lane_wait(&bars->v_empty[sv], ((vc / L::VST) & 1) ^ 1, bars))) break;
+                    mbar_arrive_expect_tx(&bars->v_full[sv], T::TILE_BYTES);
+                    for (int bx = 0; bx < T::NBOX; ++bx)
+                        tma_load_3d(sV + sv * T::TILE_BYTES + bx * T::BOX_BYTES, core ? &tmVc : &tmV,
+                                    &bars->v_full[sv], bx * 64, key0, z);
+                    ++vc;
+                }
+            }
+            // drain: every issued copy has landed before the CTA exits
+            const volatile int *never = &bars->never;
+            for (uint32_t s = 0; s < L::KST && s < kc; ++s) {
+                const uint32_t last = kc - 1 - ((kc - 1 - s) % L::KST);
+                wait_bounded(&bars->k_full[last % L::KST], (last / L::KST) & 1, never, kBwWaitNs);
+            }
+            for (uint32_t s = 0; s < L::VST && s < vc; ++s) {
+                const uint32_t last = vc - 1 - ((vc - 1 - s) % L::VST);
+                wait_bounded(&bars->v_full[last % L::VST], (last / L::VST) & 1, never, kBwWaitNs);
+            }
+            if (qc > 0) wait_bounded(&bars->q_full[0], (qc - 1) & 1, never, kBwWaitNs);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s_bf = idesc_f32acc(128, 128, true, false, false);
+            constexpr uint32_t id_s_h = idesc_f32acc(128, 128, false, false, false);
+            constexpr uint32_t id_q_bf = idesc_f32acc(128, D, true, false, true);
+            constexpr uint32_t id_q_h = idesc_f32acc(128, D, false, false, true);
+            const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+            const uint64_t dO = smem_desc_sw128(smem_addr(sO), 16, 1024);
+            const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
+            const uint64_t dkm = smem_desc_sw128(smem_addr(sK), T::BOX_BYTES, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(sV), 16, 1024);
+            constexpr uint32_t kTile16 = T::TILE_BYTES >> 4;
+            uint32_t kc = 0, vc = 0, qc = 0, it = 0;
+            int k = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
+                const QGeom G = q_geom(item, p);
+                if (!(ok = bw_lane_wait(&bars->q_full[0], qc & 1, bars))) break;
+                ++qc;
+                for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
+                    const bool core = j >= G.n_local;
+                    if (core && j == G.n_local) {
+                        // the bf16 query tiles are read: swap in the fp16 copies
+                        mma_commit(&bars->q_empty[0]);
+                        if (!(ok = bw_lane_wait(&bars->q_full[0], qc & 1, bars))) break;
+                        ++qc;
+                    }
+                    const uint32_t s = kc % L::KST, sv = vc % L::VST;
+                    if (!(ok = bw_lane_wait(&bars->k_full[s], (kc / L::KST) & 1, bars))) break;
+                    if (!(ok = bw_lane_wait(&bars->v_full[sv], (vc / L::VST) & 1, bars))) break;
+                    if (it > 0 && !(ok = bw_lane_wait(&bars->s_free, (it - 1) & 1, bars))) break;
+                    tc_fence_after_sync();
+                    mma_kk<D>(tmem + L::S_COL, dq, dk + s * kTile16, core ? id_s_h : id_s_bf);
+                    mma_kk<D>(tmem + L::DP_COL, dO, dv + sv * kTile16, core ? id_s_h : id_s_bf);
+                    mma_commit(&bars->s_full);
+                    mma_commit(&bars->v_empty[sv]);
+                    ++vc;
+                    if (!(ok = bw_lane_wait(&bars->p_full, it & 1, bars))) break;
+                    if (j == 0 && k > 0 && !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
+                        break;
+                    tc_fence_after_sync();
+                    mma_tm(tmem + L::DQ_COL, tmem + L::DS_COL, dkm + s * kTile16,
+                           core ? id_q_h : id_q_bf, j == 0);
+                    mma_commit(&bars->mm_done);
+                    mma_commit(&bars->k_empty[s]);
+                    ++kc;
+                }
+                if (!ok) break;
+                mma_commit(&bars->q_empty[0]);
+            }
+            mma_commit(&bars->drain);
+            wait_bounded(&bars->drain, 0, &bars->never, kBwWaitNs);
+        }
+    } else {
+        // ------------------------------------------------ dS warps
+        const int row = threadIdx.x & 127;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const QGeom G = q_geom(item, p);
+            const int t = G.t0 + row;
+            const bool valid = t < p.T;
+            const int64_t qrow = (static_cast<int64_t>(G.b) * p.Hq + G.hq) * p.T + t;
+            const float lse = valid ? p.lse[qrow] : 0.f;
+            const float dd = valid ? p.Dv[qrow] : 0.f;
+            const int ws_t = ws_of(t, p.g, p.w);
+            const int nc_t = ws_t / p.g;
+            for (int j = 0; j < G.n_tiles; ++j, ++it) {
+                if (!(ok = bw_warp_wait(&bars->s_full, it & 1, bars))) break;
+                tc_fence_after_sync();
+                const bool core = j >= G.n_local;
+                const int key0 = core ? (j - G.n_local) * 128 : G.ws_lo + j * 128;
+                const int lo = core ? 0 : ws_t, hi = core ? nc_t - 1 : t;
+                uint32_t pk[4][16];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t us[32], ud[32];
+                    tmem_ld32(tmem + lane_off + L::S_COL + c * 32, us);
+                    tmem_ld32(tmem + lane_off + L::DP_COL + c * 32, ud);
+                    tmem_wait_ld_dep(us);
+                    tmem_wait_ld_dep(ud);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        const int key = key0 + c * 32 + e;
+                        const bool v0 = valid && key >= lo && key <= hi;
+                        const bool v1 = valid && key + 1 >= lo && key + 1 <= hi;
+                        const float p0 = v0 ? fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - lse) : 0.f;
+                        const float p1 = v1 ? fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - lse) : 0.f;
+                        pk[c][e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - dd),
+                                              p1 * (__uint_as_float(ud[e + 1]) - dd), core);
+                    }
+                }
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->s_free);
+                // the previous tile's dQ product has read dS
+                if (it > 0) {
+                    if (!(ok = bw_warp_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
+                    tc_fence_after_sync();
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) tmem_st16(tmem + lane_off + L::DS_COL + c * 16, pk[c]);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full);
+            }
+            if (!ok) break;
+            // epilogue: dQ = (sum dS K) / sqrt(d)
+            if (!(ok = bw_warp_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
+            tc_fence_after_sync();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t u[32];
+                tmem_ld32_wait(tmem + lane_off + L::DQ_COL + c * 32, u);
+                if (valid) {
+                    float4 *dst = reinterpret_cast<float4 *>(p.dQ + qrow * D + c * 32);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        dst[q] = make_float4(__uint_as_float(u[4 * q]) * p.scale,
+                                             __uint_as_float(u[4 * q + 1]) * p.scale,
+                                             __uint_as_float(u[4 * q + 2]) * p.scale,
+                                             __uint_as_float(u[4 * q + 3]) * p.scale);
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// 3. dK, dV (raw) and dKc, dVc (core) --------------------------------------
+//
+// Work item: one 128-key tile of one (batch, kv head) and a range of query
+// tiles, for all r query heads of the kv head.  Core tiles come first, their
+// query range (every later query sees a core key) cut into chunks of
+// kCoreChunk tiles whose results are added into fp32 dKc, dVc; raw tiles
+// take every query tile that sees one of their keys and store dK, dV.
+// Warps 0-3: one key row per thread; warp 4: TMA producer; warp 5: issuer.
+// TMEM: S^T [0,128) then P^T over its first 64 columns; dP^T [128,256) then
+// dS^T over its first 64; dK [256, 256+D); dV [256+D, 256+2D).
+template <int D>
+struct BkLayout {
+    using T = Bt<D>;
+    static constexpr int QST = 2;
+    static constexpr int OFF_K = 0, OFF_V = T::TILE_BYTES;
+    static constexpr int OFF_Q = 2 * T::TILE_BYTES;                 // QST stages
+    static constexpr int OFF_O = OFF_Q + QST * T::TILE_BYTES;       // QST stages
+    static constexpr int OFF_COL = OFF_O + QST * T::TILE_BYTES;     // per-column data
+    static constexpr int OFF_BAR = OFF_COL + 2 * 3 * 128 * 4;
+    static constexpr int SMEM = OFF_BAR + 512 + 1024;
+    static constexpr uint32_t ST_COL = 0, DPT_COL = 128, DK_COL = 256, DV_COL = 256 + D;
+};
+
+struct KGeom {
+    bool core;
+    int b, h, kt;   // key tile (raw: rows 128 kt..; core: groups 128 kt..)
+    int qa, qb;     // query tiles [qa, qb)
+};
+
+// First query tile with a query that attends to core group j: query t sees
+// group j iff j < ws(t) / g, i.e. t >= (j + 1) g + w.
+__device__ __forceinline__ int core_first_qt(int j, const BwParams &p)
+{
+    return static_cast<int>((static_cast<int64_t>(j + 1) * p.g + p.w) / 128);
+}
+
+__device__ __forceinline__ KGeom k_geom(int item, const BwParams &p)
+{
+    KGeom G;
+    const int pairs = p.B * p.Hkv;
+    if (item < p.n_core_items) {
+        int u = item;
+        for (int ct = 0; ct < p.n_ct; ++ct) {
+            const int qs = core_first_qt(ct * 128, p);
+            const int nch = qs < p.n_qt ? (p.n_qt - qs + kCoreChunk - 1) / kCoreChunk : 0;
+            if (u < nch * pairs) {
+                const int chunk = u / pairs, pair = u - chunk * pairs;
+                G.core = true;
+                G.b = pair / p.Hkv;
+                G.h = pair - G.b * p.Hkv;
+                G.kt = ct;
+                G.qa = qs + chunk * kCoreChunk;
+                G.qb = min(G.qa + kCoreChunk, p.n_qt);
+                return G;
+            }
+            u -= nch * pairs;
+        }
+    }
+    const int u = item - p.n_core_items;
+    const int kt = u / pairs, pair = u - kt * pairs;
+    G.core = false;
+    G.b = pair / p.Hkv;
+    G.h = pair - G.b * p.Hkv;
+    G.kt = kt;
+    // key k is seen by queries k .. (floor(k / g) + 1) g + w - 1
+    const int klast = min(kt * 128 + 127, p.T - 1);
+    const int tmax = min((klast / p.g + 1) * p.g + p.w - 1, p.T - 1);
+    G.qa = kt;
+    G.qb = tmax / 128 + 1;
+    return G;
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+    bw_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
+                  const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
+                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                  const __grid_constant__ CUtensorMap tmKc, const __grid_constant__ CUtensorMap tmVc,
+                  const BwParams p)
+{
+    using L = BkLayout<D>;
+    using T = Bt<D>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t *sK = smem + L::OFF_K, *sV = smem + L::OFF_V;
+    uint8_t *sQ = smem + L::OFF_Q, *sO = smem + L::OFF_O;
+    float *col = reinterpret_cast<float *>(smem + L::OFF_COL);  // [2][3][128]: lse, D, ws
+    BwBars *bars = reinterpret_cast<BwBars *>(smem + L::OFF_BAR);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int n_items = p.n_items;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L::QST; ++s) {
+            mbar_init(&bars->q_full[s], 1);
+            mbar_init(&bars->q_empty[s], 1);
+        }
+        mbar_init(&bars->kv_full, 1);
+        mbar_init(&bars->kv_empty, 1);
+        mbar_init(&bars->s_full, 1);
+        mbar_init(&bars->p_full, 4);
+        mbar_init(&bars->mm_done, 1);
+        mbar_init(&bars->acc_empty, 4);
+        mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        bars->never = 0;
+        mbar_fence_init();
+    }
+    if (warp == 4) {
+        tmem_alloc(&bars->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+
+    if (warp == 4) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            uint32_t qc = 0, kvc = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+                const KGeom G = k_geom(item, p);
+                const int z = G.b * p.Hkv + G.h;
+                if (kvc > 0 && !(ok = bw_lane_wait(&bars->kv_empty, (kvc - 1) & 1, bars))) break;
+                mbar_arrive_expect_tx(&bars->kv_full, 2 * T::TILE_BYTES);
+                for (int bx = 0; bx < T::NBOX; ++bx) {
+                    tma_load_3d(sK + bx * T::BOX_BYTES, G.core ? &tmKc : &tmK, &bars->kv_full,
+                                bx * 64, G.kt * 128, z);
+                    tma_load_3d(sV + bx * T::BOX_BYTES, G.core ? &tmVc : &tmV, &bars->kv_full,
+                                bx * 64, G.kt * 128, z);
+                }
+                ++kvc;
+                for (int kh = 0; ok && kh < p.r; ++kh) {
+                    const int zq = G.b * p.Hq + G.h * p.r + kh;
+                    for (int qt = G.qa; qt < G.qb; ++qt) {
+                        const int s = qc % L::QST;
+                        if (!(ok = bw_lane_wait(&bars->q_empty[s], ((qc / L::QST) & 1) ^ 1, bars)))
+                            break;
+                        mbar_arrive_expect_tx(&bars->q_full[s], 2 * T::TILE_BYTES);
+                        for (int bx = 0; bx < T::NBOX; ++bx) {
+                            tma_load_3d(sQ + s * T::TILE_BYTES + bx * T::BOX_BYTES,
+                                        G.core ? &tmQ16 : &tmQ, &bars->q_full[s], bx * 64,
+                                        qt * 128, zq);
+                            tma_load_3d(sO + s * T::TILE_BYTES + bx * T::BOX_BYTES,
+                                        G.core ? &tmO16 : &tmO, &bars->q_full[s], bx * 64,
+                                        qt * 128, zq);
+                        }
+                        ++qc;
+                    }
+                }
+            }
+            const volatile int *never = &bars->never;
+            for (uint32_t s = 0; s < L::QST && s < qc; ++s) {
+                const uint32_t last = qc - 1 - ((qc - 1 - s) % L::QST);
+                wait_bounded(&bars->q_full[last % L::QST], (last / L::QST) & 1, never, kBwWaitNs);
+            }
+            if (kvc > 0) wait_bounded(&bars->kv_full, (kvc - 1) & 1, never, kBwWaitNs);
+        }
+    } else if (warp == 5) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id_s_bf = idesc_f32acc(128, 128, true, false, false);
+            constexpr uint32_t id_s_h = idesc_f32acc(128, 128, false, false, false);
+            constexpr uint32_t id_a_bf = idesc_f32acc(128, D, true, false, true);
+            constexpr uint32_t id_a_h = idesc_f32acc(128, D, false, false, true);
+            const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
+            const uint64_t dv = smem_desc_sw128(smem_addr(sV), 16, 1024);
+            const uint64_t dq = smem_desc_sw128(smem_addr(sQ), 16, 1024);
+            const uint64_t dqm = smem_desc_sw128(smem_addr(sQ), T::BOX_BYTES, 1024);
+            const uint64_t dO = smem_desc_sw128(smem_addr(sO), 16, 1024);
+            const uint64_t dOm = smem_desc_sw128(smem_addr(sO), T::BOX_BYTES, 1024);
+            constexpr uint32_t kTile16 = T::TILE_BYTES >> 4;
+            uint32_t qc = 0, it = 0, kvc = 0;
+            int k = 0;
+            bool ok = true;
+            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
+                const KGeom G = k_geom(item, p);
+                const uint32_t ids = G.core ? id_s_h : id_s_bf, ida = G.core ? id_a_h : id_a_bf;
+                if (!(ok = bw_lane_wait(&bars->kv_full, kvc & 1, bars))) break;
+                ++kvc;
+                const int n_tiles = p.r * (G.qb - G.qa);
+                for (int i = 0; ok && i < n_tiles; ++i, ++it) {
+                    const uint32_t s = qc % L::QST;
+                    if (!(ok = bw_lane_wait(&bars->q_full[s], (qc / L::QST) & 1, bars))) break;
+                    // the previous tile's dV, dK products have read P^T, dS^T
+                    if (it > 0 && !(ok = bw_lane_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
+                    tc_fence_after_sync();
+                    mma_kk<D>(tmem + L::ST_COL, dk, dq + s * kTile16, ids);
+                    mma_kk<D>(tmem + L::DPT_COL, dv, dO + s * kTile16, ids);
+                    mma_commit(&bars->s_full);
+                    if (!(ok = bw_lane_wait(&bars->p_full, it & 1, bars))) break;
+                    if (i == 0 && k > 0 && !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
+                        break;
+                    tc_fence_after_sync();
+                    mma_tm(tmem + L::DV_COL, tmem + L::ST_COL, dOm + s * kTile16, ida, i == 0);
+                    mma_tm(tmem + L::DK_COL, tmem + L::DPT_COL, dqm + s * kTile16, ida, i == 0);
+                    mma_commit(&bars->mm_done);
+                    mma_commit(&bars->q_empty[s]);
+                    ++qc;
+                }
+                if (!ok) break;
+                mma_commit(&bars->kv_empty);
+            }
+            mma_commit(&bars->drain);
+            wait_bounded(&bars->drain, 0, &bars->never, kBwWaitNs);
+        }
+    } else {
+        // ------------------------------------------------ P^T, dS^T warps
+        const int row = threadIdx.x & 127;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        uint32_t it = 0;
+        bool ok = true;
+        for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x) {
+            const KGeom G = k_geom(item, p);
+            const int key = G.kt * 128 + row;  // raw key, or core group
+            const bool kvalid = G.core ? key < p.m : key < p.T;
+            const int n_tiles = p.r * (G.qb - G.qa);
+            for (int i = 0; i < n_tiles; ++i, ++it) {
+                const int kh = i / (G.qb - G.qa), qt = G.qa + (i - kh * (G.qb - G.qa));
+                const int hq = G.h * p.r + kh;
+                // per-column data of this query tile: log-sum-exp, D, window
+                // start (or core count), staged in shared memory
+                float *cb = col + (it & 1) * 3 * 128;
+                {
+                    const int t = qt * 128 + row;
+                    const int64_t qrow = (static_cast<int64_t>(G.b) * p.Hq + hq) * p.T + t;
+                    const bool tv = t < p.T;
+                    const int wst = ws_of(t, p.g, p.w);
+                    cb[row] = tv ? p.lse[qrow] : 0.f;
+                    cb[128 + row] = tv ? p.Dv[qrow] : 0.f;
+                    // raw: the lowest key t sees; core: the number of groups
+                    // it sees; a query past the end sees nothing
+                    cb[256 + row] = __int_as_float(tv ? (G.core ? wst / p.g : wst) : (G.core ? 0 : 1 << 30));
+                }
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (!(ok = bw_warp_wait(&bars->s_full, it & 1, bars))) break;
+                tc_fence_after_sync();
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    uint32_t us[32], ud[32], pp[16], pd[16];
+                    tmem_ld32(tmem + lane_off + L::ST_COL + c * 32, us);
+                    tmem_ld32(tmem + lane_off + L::DPT_COL + c * 32, ud);
+                    tmem_wait_ld_dep(us);
+                    tmem_wait_ld_dep(ud);
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+                        float pv[2], dsv[2];
+#pragma unroll
+                        for (int x = 0; x < 2; ++x) {
+                            const int cc = c * 32 + e + x;
+                            const int t = qt * 128 + cc;
+                            const int lim = __float_as_int(cb[256 + cc]);
+                            const bool vis = kvalid && (G.core ? key < lim : (key >= lim && key <= t));
+                            const float pr = vis ? fast_exp2(__uint_as_float(us[e + x]) * p.scale_log2 - cb[cc]) : 0.f;
+                            pv[x] = pr;
+                            dsv[x] = pr * (__uint_as_float(ud[e + x]) - cb[128 + cc]);
+                        }
+                        pp[e / 2] = pack16(pv[0], pv[1], G.core);
+                        pd[e / 2] = pack16(dsv[0], dsv[1], G.core);
+                    }
+                    // over columns this thread has already read
+                    tmem_st16(tmem + lane_off + L::ST_COL + c * 16, pp);
+                    tmem_st16(tmem + lane_off + L::DPT_COL + c * 16, pd);
+                }
+                tmem_wait_st();
+                tc_fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&bars->p_full);
+            }
+            if (!ok) break;
+            // epilogue: dK = (sum dS^T Q) / sqrt(d), dV = sum P^T dO
+            if (!(ok = bw_warp_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
+            tc_fence_after_sync();
+            const int64_t krow = (static_cast<int64_t>(G.b) * p.Hkv + G.h) * (G.core ? p.m : p.T) + key;
+            float *dKo = (G.core ? p.dKc : p.dK) + krow * D;
+            float *dVo = (G.core ? p.dVc : p.dV) + krow * D;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t uk[32], uv[32];
+                tmem_ld32_wait(tmem + lane_off + L::DK_COL + c * 32, uk);
+                tmem_ld32_wait(tmem + lane_off + L::DV_COL + c * 32, uv);
+                if (!kvalid) continue;
+                if (G.core) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        atomicAdd(dKo + c * 32 + e, __uint_as_float(uk[e]) * p.scale);
+                        atomicAdd(dVo + c * 32 + e, __uint_as_float(uv[e]));
+                    }
+                } else {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        reinterpret_cast<float4 *>(dKo + c * 32)[q] =
+                            make_float4(__uint_as_float(uk[4 * q]) * p.scale,
+                                        __uint_as_float(uk[4 * q + 1]) * p.scale,
+                                        __uint_as_float(uk[4 * q + 2]) * p.scale,
+                                        __uint_as_float(uk[4 * q + 3]) * p.scale);
+                        reinterpret_cast<float4 *>(dVo + c * 32)[q] =
+                            make_float4(__uint_as_float(uv[4 * q]), __uint_as_float(uv[4 * q + 1]),
+                                        __uint_as_float(uv[4 * q + 2]), __uint_as_float(uv[4 * q + 3]));
+                    }
+                }
+            }
+            tc_fence_before_sync();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bars->acc_empty);
+        }
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 4) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// 4. The pooling's chain rule ------------------------------------------------
+//
+// One warp per (batch, kv head, group j), lane l owning dims l*DPL ..: with
+// the group's keys Kg, values Vg, the r scoring queries q_k (token jg+g-1)
+// and softmax vectors s_k = softmax(Kg q_k / sqrt(d)), a = mean_k s_k:
+//   dK_g += a dKc,  dV_g += a dVc,  da = Kg dKc + Vg dVc,
+//   per head k: dz = s_k (da/r - s_k . da/r),
+//   dq_k += (sum_i dz_i Kg_i) / sqrt(d),  dK_g += dz q_k / sqrt(d).
+template <int D>
+__global__ void bw_pool_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
+                               const uint16_t *__restrict__ V, const BwParams p)
+{
+    constexpr int DPL = D / 32;
+    extern __shared__ float pool_bw_smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int nwarp = blockDim.x >> 5;
+    float *sc = pool_bw_smem + warp * (p.r + 1) * p.g;  // [r][g] softmax, then [g] da
+    const int64_t n_groups = static_cast<int64_t>(p.B) * p.Hkv * p.m;
+    for (int64_t gid = static_cast<int64_t>(blockIdx.x) * nwarp + warp; gid < n_groups;
+         gid += static_cast<int64_t>(gridDim.x) * nwarp) {
+        const int64_t pair = gid / p.m, j = gid - pair * p.m;
+        const int64_t b = pair / p.Hkv, h = pair - b * p.Hkv;
+        const int64_t row0 = pair * p.T + j * p.g;  // first key row of the group
+        const int64_t last = j * p.g + p.g - 1;
+        float dkc[DPL], dvc[DPL];
+#pragma unroll
+        for (int e = 0; e < DPL; ++e) {
+            dkc[e] = p.dKc[(pair * p.m + j) * D + lane * DPL + e];
+            dvc[e] = p.dVc[(pair * p.m + j) * D + lane * DPL + e];
+        }
+        // scores and softmax per query head
+        for (int k = 0; k < p.r; ++k) {
+            const uint16_t *q = Q + ((b * p.Hq + h * p.r + k) * p.T + last) * D + lane * DPL;
+            float qf[DPL];
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) qf[e] = __uint_as_float(static_cast<uint32_t>(q[e]) << 16);
+            float mx = -INFINITY;
+            for (int i = 0; i < p.g; ++i) {
+                const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
+                float s = 0.f;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e)
+                    s = fmaf(qf[e], __uint_as_float(static_cast<uint32_t>(kr[e]) << 16), s);
+                s = warp_sum(s) * p.scale_log2;
+                if (lane == 0) sc[k * p.g + i] = s;
+                mx = fmaxf(mx, s);
+            }
+            __syncwarp();
+            float sum = 0.f;
+            for (int i = lane; i < p.g; i += 32) {
+                const float e = exp2f(sc[k * p.g + i] - mx);
+                sc[k * p.g + i] = e;
+                sum += e;
+            }
+            sum = warp_sum(sum);
+            __syncwarp();
+            for (int i = lane; i < p.g; i += 32) sc[k * p.g + i] /= sum;
+            __syncwarp();
+        }
+        // dK_g, dV_g through the weights; da_i
+        float *da = sc + p.r * p.g;
+        const float inv_r = 1.0f / static_cast<float>(p.r);
+        for (int i = 0; i < p.g; ++i) {
+            float a = 0.f;
+            for (int k = 0; k < p.r; ++k) a += sc[k * p.g + i];
+            a *= inv_r;
+            const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
+            const uint16_t *vr = V + (row0 + i) * D + lane * DPL;
+            float *dkr = p.dK + (row0 + i) * D + lane * DPL;
+            float *dvr = p.dV + (row0 + i) * D + lane * DPL;
+            float s = 0.f;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) {
+                s = fmaf(__uint_as_float(static_cast<uint32_t>(kr[e]) << 16), dkc[e], s);
+                s = fmaf(__uint_as_float(static_cast<uint32_t>(vr[e]) << 16), dvc[e], s);
+                dkr[e] += a * dkc[e];
+                dvr[e] += a * dvc[e];
+            }
+            s = warp_sum(s);
+            if (lane == 0) da[i] = s * inv_r;
+        }
+        __syncwarp();
+        // through each head's softmax to its query and the keys
+        for (int k = 0; k < p.r; ++k) {
+            float sd = 0.f;
+            for (int i = lane; i < p.g; i += 32) sd += sc[k * p.g + i] * da[i];
+            sd = warp_sum(sd);
+            const int64_t qrow = (b * p.Hq + h * p.r + k) * p.T + last;
+            const uint16_t *q = Q + qrow * D + lane * DPL;
+            float dq[DPL];
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) dq[e] = 0.f;
+            for (int i = 0; i < p.g; ++i) {
+                const float dz = sc[k * p.g + i] * (da[i] - sd);
+                const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
+                float *dkr = p.dK + (row0 + i) * D + lane * DPL;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) {
+                    dq[e] = fmaf(dz, __uint_as_float(static_cast<uint32_t>(kr[e]) << 16), dq[e]);
+                    dkr[e] += dz * p.scale * __uint_as_float(static_cast<uint32_t>(q[e]) << 16);
+                }
+            }
+            float *dqr = p.dQ + qrow * D + lane * DPL;
+#pragma unroll
+            for (int e = 0; e < DPL; ++e) dqr[e] += dq[e] * p.scale;
+        }
+        __syncwarp();
+    }
+}
+
+template <int D>
+cudaError_t launch_bw(const void *Q, const void *K, const void *V, const void *Kc,
+                      const void *Vc, const void *O, bool o_f32, const float *lse,
+                      const void *dO, float *dQ, float *dK, float *dV, int B, int Hq, int Hkv,
+                      int64_t T, int g, int w, void *workspace, cudaStream_t s)
+{
+    const int64_t m = T / g;
+    const int64_t rows = static_cast<int64_t>(B) * Hq * T;
+    BwLayoutHost L = bw_layout(B, Hq, Hkv, T, D, g);
+    char *ws = static_cast<char *>(workspace);
+    uint16_t *Q16 = reinterpret_cast<uint16_t *>(ws + L.q16);
+    uint16_t *dO16 = reinterpret_cast<uint16_t *>(ws + L.do16);
+    float *Dv = reinterpret_cast<float *>(ws + L.dv);
+    float *dKc = reinterpret_cast<float *>(ws + L.dkc);
+    float *dVc = reinterpret_cast<float *>(ws + L.dvc);
+
+    BwParams p;
+    p.B = B;
+    p.Hq = Hq;
+    p.Hkv = Hkv;
+    p.r = Hq / Hkv;
+    p.T = static_cast<int>(T);
+    p.g = g;
+    p.w = w;
+    p.m = static_cast<int>(m);
+    p.scale = 1.0f / sqrtf(static_cast<float>(D));
+    p.scale_log2 = kLog2e * p.scale;
+    p.lse = lse;
+    p.Dv = Dv;
+    p.dQ = dQ;
+    p.dK = dK;
+    p.dV = dV;
+    p.dKc = dKc;
+    p.dVc = dVc;
+    p.n_qt = static_cast<int>((T + 127) / 128);
+    p.n_kt = p.n_qt;
+    p.n_ct = static_cast<int>((m + 127) / 128);
+    int core_items = 0;
+    for (int ct = 0; ct < p.n_ct; ++ct) {
+        const int qs = static_cast<int>((static_cast<int64_t>(ct * 128 + 1) * g + w) / 128);
+        if (qs < p.n_qt) core_items += (p.n_qt - qs + kCoreChunk - 1) / kCoreChunk;
+    }
+    p.n_core_items = core_items * B * Hkv;
+    p.n_items = p.n_core_items + p.n_kt * B * Hkv;
+
+    cudaError_t e = cudaSuccess;
+    if (m > 0) {
+        e = cudaMemsetAsync(ws + L.dkc, 0, L.dvc + L.dvc_bytes - L.dkc, s);
+        if (e != cudaSuccess) return e;
+    }
+    // 1. D and the fp16 copies
+    {
+        const int threads = 256;
+        const int64_t want = (rows * 32 + threads - 1) / threads;
+        const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
+        if (o_f32)
+            bw_prep_kernel<D, true><<<blocks, threads, 0, s>>>(
+                static_cast<const uint16_t *>(dO), O, static_cast<const uint16_t *>(Q), Dv, Q16,
+                dO16, rows);
+        else
+            bw_prep_kernel<D, false><<<blocks, threads, 0, s>>>(
+                static_cast<const uint16_t *>(dO), O, static_cast<const uint16_t *>(Q), Dv, Q16,
+                dO16, rows);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    CUtensorMap mQ, mO, mQ16, mO16, mK, mV, mKc, mVc;
+    const int64_t pq = static_cast<int64_t>(B) * Hq, pk = static_cast<int64_t>(B) * Hkv;
+    bool ok = make_map(&mQ, Q, D, T, pq) && make_map(&mO, dO, D, T, pq) &&
+              make_map(&mQ16, Q16, D, T, pq, true) && make_map(&mO16, dO16, D, T, pq, true) &&
+              make_map(&mK, K, D, T, pk) && make_map(&mV, V, D, T, pk);
+    if (m > 0)
+        ok = ok && make_map(&mKc, Kc, D, m, pk, true) && make_map(&mVc, Vc, D, m, pk, true);
+    else {
+        mKc = mK;
+        mVc = mV;
+    }
+    if (!ok) return cudaErrorInvalidValue;
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // 2. dQ (attention part)
+    {
+        using LQ = BqLayout<D>;
+        const int items = p.n_qt * B * Hq;
+        const int grid = items < sms ? items : sms;
+        if ((e = cudaFuncSetAttribute(bw_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      LQ::SMEM)) != cudaSuccess)
+            return e;
+        bw_dq_kernel<D><<<grid, 192, LQ::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc, mVc, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // 3. dK, dV and dKc, dVc
+    {
+        using LK = BkLayout<D>;
+        const int grid = p.n_items < sms ? p.n_items : sms;
+        if ((e = cudaFuncSetAttribute(bw_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      LK::SMEM)) != cudaSuccess)
+            return e;
+        bw_dkv_kernel<D><<<grid, 192, LK::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc, mVc, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    // 4. the pooling
+    if (m > 0) {
+        const int warps = 8;
+        const size_t smem = sizeof(float) * warps * (p.r + 1) * g;
+        const int64_t groups = static_cast<int64_t>(B) * Hkv * m;
+        const int64_t want = (groups + warps - 1) / warps;
+        const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);
+        if (smem > 48 * 1024 &&
+            (e = cudaFuncSetAttribute(bw_pool_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                      static_cast<int>(smem))) != cudaSuccess)
+            return e;
+        bw_pool_kernel<D><<<blocks, warps * 32, smem, s>>>(
+            static_cast<const uint16_t *>(Q), static_cast<const uint16_t *>(K),
+            static_cast<const uint16_t *>(V), p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+BwLayoutHost bw_layout(int B, int Hq, int Hkv, int64_t T, int d, int g)
+{
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    const size_t qd = static_cast<size_t>(B) * Hq * T * d * 2;
+    const size_t rows = static_cast<size_t>(B) * Hq * T * 4;
+    const size_t core = static_cast<size_t>(B) * Hkv * (T / g) * d * 4;
+    BwLayoutHost L;
+    L.q16 = 0;
+    L.do16 = L.q16 + up(qd);
+    L.dv = L.do16 + up(qd);
+    L.dkc = L.dv + up(rows);
+    L.dvc = L.dkc + up(core);
+    L.dvc_bytes = up(core);
+    L.total = L.dvc + L.dvc_bytes;
+    return L;
+}
+
+cudaError_t launch_backward(const void *Q, const void *K, const void *V, const void *Kc,
+                            const void *Vc, const void *O, bool o_f32, const float *lse,
+                            const void *dO, float *dQ, float *dK, float *dV, int B, int Hq,
+                            int Hkv, int64_t T, int d, int g, int w, void *workspace,
+                            cudaStream_t s)
+{
+    if (T == 0) return cudaSuccess;
+    if (d == 128)
+        return launch_bw<128>(Q, K, V, Kc, Vc, O, o_f32, lse, dO, dQ, dK, dV, B, Hq, Hkv, T, g,
+                              w, workspace, s);
+    return launch_bw<64>(Q, K, V, Kc, Vc, O, o_f32, lse, dO, dQ, dK, dV, B, Hq, Hkv, T, g, w,
+                         workspace, s);
+}
+
+cudaError_t backward_status_read_clear(unsigned int *v)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(v, g_backward_status, sizeof(*v));
+    if (e == cudaSuccess && *v) e = cudaMemcpyToSymbol(g_backward_status, &zero, sizeof(zero));
+    return e;
+}
+
+}  // namespace cca

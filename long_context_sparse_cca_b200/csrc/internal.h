@@ -59,10 +59,25 @@ cudaError_t launch_decode_step(void *k_core, void *v_core, void *k_tail, void *v
                                cudaStream_t s);
 
 // Fused core + local attention over a whole sequence (tcgen05 kernel).
+// lse != nullptr: also write each row's log-sum-exp (log2 units), fp32
+// [B, Hq, T], for the backward pass.
 cudaError_t launch_prefill(const void *Q, const void *K, const void *V,
                            const void *Kc, const void *Vc, void *O, bool o_f32,
                            int B, int Hq, int Hkv, int64_t T, int d, int g,
-                           int w, cudaStream_t s);
+                           int w, cudaStream_t s, float *lse = nullptr);
+
+// Backward pass (training).  Workspace layout (byte offsets, 256-aligned):
+// fp16 copies of Q and dO, D = rowsum(dO * O), fp32 dKc and dVc.
+struct BwLayoutHost {
+    size_t q16, do16, dv, dkc, dvc, dvc_bytes, total;
+};
+BwLayoutHost bw_layout(int B, int Hq, int Hkv, int64_t T, int d, int g);
+cudaError_t launch_backward(const void *Q, const void *K, const void *V, const void *Kc,
+                            const void *Vc, const void *O, bool o_f32, const float *lse,
+                            const void *dO, float *dQ, float *dK, float *dV, int B, int Hq,
+                            int Hkv, int64_t T, int d, int g, int w, void *workspace,
+                            cudaStream_t s);
+cudaError_t backward_status_read_clear(unsigned int *v);
 
 // Device status words (bits kStatusTimeout, kStatusRange): read and clear.
 cudaError_t prefill_status_read_clear(unsigned int *v);

@@ -45,6 +45,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include "tma_map.h"
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -84,6 +86,7 @@ struct Params {
     float scale_log2;
     void *O;
     int o_f32;
+    float *lse;  // [B, Hq, T]: log2 of each row's softmax denominator (LSE instance)
 };
 
 __device__ __forceinline__ int ws_of(int t, int g, int w)
@@ -213,7 +216,10 @@ __device__ __forceinline__ float row_max128(const float (&x)[128])
     return fmax3(fmax3(m[0], m[1], m[2]), fmax3(m[3], m[4], m[5]), fmaxf(m[6], m[7]));
 }
 
-template <int D>
+// LSE: also write each row's log-sum-exp (log2 units: log2 of the sum of
+// 2^(logit / ln 2) over the row's keys), which the backward kernels need;
+// a separate instance, so that the inference kernel is unchanged.
+template <int D, bool LSE>
 __global__ void __launch_bounds__(352, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
@@ -576,6 +582,7 @@ __global__ void __launch_bounds__(352, 1)
             const float inv = 1.0f / l_run;
             const int64_t orow = (static_cast<int64_t>(G.b) * p.Hq + G.hq) * p.T + t;
             const bool store = t < p.T;
+            if (LSE && store) p.lse[orow] = (m_run == -INFINITY ? 0.f : m_run) + __log2f(l_run);
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float o[32];
@@ -615,46 +622,10 @@ __global__ void __launch_bounds__(352, 1)
     }
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (!fn) {
-        cudaDriverEntryPointQueryResult q;
-        void *f = nullptr;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
-    }
-    return fn;
-}
-
-// 3-D map over a [planes, rows, d] tensor of 16-bit elements (bf16 or
-// fp16), 64 x 128 x 1 boxes, 128-byte swizzle, zero fill outside the tensor.
-bool make_map(CUtensorMap *m, const void *ptr, int d, int64_t rows, int64_t planes,
-              bool f16 = false)
-{
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows),
-                          static_cast<cuuint64_t>(planes)};
-    cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                             static_cast<cuuint64_t>(rows) * d * 2};
-    cuuint32_t box[3] = {64, 128, 1};
-    cuuint32_t estr[3] = {1, 1, 1};
-    const CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16
-                                 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
-                          3, const_cast<void *>(ptr),
-                          dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
-}
-
 template <int D>
 cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc,
                      const void *Vc, void *O, bool o_f32, int B, int Hq, int Hkv,
-                     int64_t T, int g, int w, cudaStream_t s)
+                     int64_t T, int g, int w, cudaStream_t s, float *lse)
 {
     using C = Pf<D>;
     CUtensorMap mQ, mK, mV, mKc, mVc;
@@ -684,14 +655,16 @@ cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc
     p.scale_log2 = kLog2e / sqrtf(static_cast<float>(D));
     p.O = O;
     p.o_f32 = o_f32 ? 1 : 0;
+    p.lse = lse;
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = p.n_items < sms ? p.n_items : sms;
-    cudaError_t e = cudaFuncSetAttribute(prefill_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    auto kern = lse ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM);
     if (e != cudaSuccess) return e;
-    prefill_kernel<D><<<grid, C::THREADS, C::SMEM, s>>>(mQ, mK, mV, mKc, mVc, p);
+    kern<<<grid, C::THREADS, C::SMEM, s>>>(mQ, mK, mV, mKc, mVc, p);
     return cudaGetLastError();
 }
 
@@ -700,11 +673,11 @@ cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc
 cudaError_t launch_prefill(const void *Q, const void *K, const void *V,
                            const void *Kc, const void *Vc, void *O, bool o_f32,
                            int B, int Hq, int Hkv, int64_t T, int d, int g,
-                           int w, cudaStream_t s)
+                           int w, cudaStream_t s, float *lse)
 {
     if (T == 0) return cudaSuccess;
-    if (d == 128) return launch_d<128>(Q, K, V, Kc, Vc, O, o_f32, B, Hq, Hkv, T, g, w, s);
-    return launch_d<64>(Q, K, V, Kc, Vc, O, o_f32, B, Hq, Hkv, T, g, w, s);
+    if (d == 128) return launch_d<128>(Q, K, V, Kc, Vc, O, o_f32, B, Hq, Hkv, T, g, w, s, lse);
+    return launch_d<64>(Q, K, V, Kc, Vc, O, o_f32, B, Hq, Hkv, T, g, w, s, lse);
 }
 
 cudaError_t prefill_status_read_clear(unsigned int *v)
