@@ -109,6 +109,26 @@ def prefill_entry(wl, t: dict, pk: dict, world: int) -> dict:
     return out
 
 
+def backward_flops(wl) -> float:
+    """Algorithmic FLOPs of the attention backward: 10 d per attended
+    (query, key) pair (S recomputed, dP, dV, dK, dQ), every batch row and
+    query head; the pooling's chain rule is not counted."""
+    return 2.5 * prefill_flops(wl)
+
+
+def backward_entry(wl, t: dict, pk: dict, world: int) -> dict:
+    """Time and tensor-core fraction of the backward pass on one workload."""
+    flops = backward_flops(wl)
+    tf = flops / (t["backward_ms"] * 1e-3) / 1e12
+    return {"backward_ms": t["backward_ms"], "forward_lse_ms": t["forward_ms"],
+            "tflops": tf, "algorithmic_flops": flops,
+            "frac_burst": tf / pk["bf16_tflops"],
+            "frac_sustained": (tf / pk["bf16_tflops_sustained"]
+                               if pk["bf16_tflops_sustained"] else None),
+            "what": "cca_attn_backward: row sums + tcgen05 dQ + tcgen05 dK/dV + pooling "
+                    "chain rule; FLOPs 10 d per attended (query, key) pair"}
+
+
 def decode_bytes(wl, t: int) -> float:
     """Algorithmic bytes of one decode step at token t: every key and value
     row the token attends to, plus its query and output rows."""
@@ -398,6 +418,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         extra[name] = time_prefill(cca, synth.WORKLOADS[name], args.steps, args.warmup,
                                    stream, torch)
 
+    # --- the backward pass (training) on the 32K workload: the forward with
+    # log-sum-exp, then cca_attn_backward (four launches)
+    if do_prefill and not args.no_backward:
+        extra["backward"] = time_backward(cca, synth.PREFILL_32K, args.steps, args.warmup,
+                                          stream, torch)
+
     # one all-reduce of every timing, the same on all ranks (no e2e: -1)
     total_ms, mean_pool, mean_prefill, mean_decode, mean_e2e = max_over_ranks(
         [total_ms, float(np.mean(pool_ms)), float(np.mean(prefill_ms)),
@@ -405,14 +431,50 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         world, "cuda")
     mean_e2e = mean_e2e if mean_e2e >= 0 else None
     for name in list(extra):
-        extra[name] = dict(zip(("pool_ms", "prefill_ms"),
-                               max_over_ranks([extra[name]["pool_ms"],
-                                               extra[name]["prefill_ms"]], world, "cuda")))
+        keys = sorted(extra[name])
+        extra[name] = dict(zip(keys, max_over_ranks([extra[name][k] for k in keys], world,
+                                                    "cuda")))
     h2d = 3 * Q.numel() * 2 if do_prefill else 0
     d2h = O.numel() * 2 if do_prefill else 0
     return dict(total_ms=total_ms, pool_ms=mean_pool, prefill_ms=mean_prefill,
                 decode_ms=mean_decode, e2e_ms=mean_e2e, clocks=clk.summary(),
                 h2d=h2d, d2h=d2h, extra=extra)
+
+
+def time_backward(cca, wl, steps: int, warmup: int, stream, torch) -> dict:
+    """Mean CUDA-event times (ms) of cca_attn_prefill_lse and of
+    cca_attn_backward on one workload (synthetic upstream gradient dO,
+    N(0,1) bf16), inputs resident in HBM."""
+    x = synth.generate(wl)
+    Q, K, V = _dev(x.q, torch), _dev(x.k, torch), _dev(x.v, torch)
+    dO = _dev(synth.random_bf16(x.q.shape, wl.seed + 100), torch)
+    del x
+    Kc, Vc = cca.cca_pool(Q, K, V, wl.g)
+    O = torch.empty((wl.B, wl.Hq, wl.T, wl.d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((wl.B, wl.Hq, wl.T), dtype=torch.float32, device="cuda")
+    dQ = torch.empty((wl.B, wl.Hq, wl.T, wl.d), dtype=torch.float32, device="cuda")
+    dK = torch.empty((wl.B, wl.Hkv, wl.T, wl.d), dtype=torch.float32, device="cuda")
+    dV = torch.empty_like(dK)
+    ws = torch.empty(cca.cca_attn_backward_workspace_bytes(wl.B, wl.Hq, wl.Hkv, wl.T, wl.d,
+                                                           wl.g), dtype=torch.uint8,
+                     device="cuda")
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(warmup + steps)]
+    for e in evs:
+        e[0].record(stream)
+        cca.cca_attn_prefill_lse(Q, K, V, Kc, Vc, wl.g, wl.w, O=O, lse=lse)
+        e[1].record(stream)
+        cca.cca_attn_backward(Q, K, V, Kc, Vc, O, lse, dO, wl.g, wl.w, dQ, dK, dV, workspace=ws)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    st = cca.cca_device_status()
+    assert st == cca.CCA_OK, cca.status_string(st)
+    timed = evs[warmup:]
+    out = {"forward_ms": float(np.mean([e[0].elapsed_time(e[1]) for e in timed])),
+           "backward_ms": float(np.mean([e[1].elapsed_time(e[2]) for e in timed]))}
+    del Q, K, V, dO, Kc, Vc, O, lse, dQ, dK, dV, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def time_prefill(cca, wl, steps: int, warmup: int, stream, torch) -> dict:
@@ -572,6 +634,8 @@ def main(argv=None) -> int:
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer pass")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip timing the 32K and GQA prefill workloads")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip timing the backward pass on the 32K workload")
     args = ap.parse_args(argv)
     args.prefill_wl = synth.WORKLOADS[args.prefill_workload]
     if args.warmup < 3:
@@ -658,7 +722,10 @@ def main(argv=None) -> int:
                             "bytes": dbytes,
                             "launches": "cca_decode_step: one kernel per token (append, split-K attention, merge)"},
             **{f"prefill[{name}]": prefill_entry(synth.WORKLOADS[name], t, pk, world)
-               for name, t in r["extra"].items()},
+               for name, t in r["extra"].items() if name != "backward"},
+            **({"backward[" + synth.PREFILL_32K.name + "]": backward_entry(
+                synth.PREFILL_32K, r["extra"]["backward"], pk, world)}
+               if "backward" in r["extra"] else {}),
         },
         "kv_cache": cache_bytes(pw, pw.T),
         "clocks": r["clocks"],

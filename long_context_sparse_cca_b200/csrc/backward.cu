@@ -473,7 +473,7 @@ struct BkLayout {
     static constexpr int OFF_Q = 2 * T::TILE_BYTES;                 // QST stages
     static constexpr int OFF_O = OFF_Q + QST * T::TILE_BYTES;       // QST stages
     static constexpr int OFF_COL = OFF_O + QST * T::TILE_BYTES;     // per-column data
-    static constexpr int OFF_BAR = OFF_COL + 2 * 3 * 128 * 4;
+    static constexpr int OFF_BAR = OFF_COL + 2 * 128 * 8;
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
     static constexpr uint32_t ST_COL = 0, DPT_COL = 128, DK_COL = 256, DV_COL = 256 + D;
 };
@@ -542,7 +542,8 @@ __global__ void __launch_bounds__(192, 1)
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t *sK = smem + L::OFF_K, *sV = smem + L::OFF_V;
     uint8_t *sQ = smem + L::OFF_Q, *sO = smem + L::OFF_O;
-    float *col = reinterpret_cast<float *>(smem + L::OFF_COL);  // [2][3][128]: lse, D, ws
+    // [2][128] (lse, D) of the current query tile's columns
+    const uint32_t col_s = smem_addr(smem + L::OFF_COL);
     BwBars *bars = reinterpret_cast<BwBars *>(smem + L::OFF_BAR);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_items = p.n_items;
@@ -674,24 +675,39 @@ __global__ void __launch_bounds__(192, 1)
             const int key = G.kt * 128 + row;  // raw key, or core group
             const bool kvalid = G.core ? key < p.m : key < p.T;
             const int n_tiles = p.r * (G.qb - G.qa);
+            // the queries that see this key form one range [t_lo, t_hi]: a
+            // raw key k is seen by t = k .. (floor(k / g) + 1) g + w - 1
+            // (its window start ws(t) <= k), core group j by every
+            // t >= (j + 1) g + w (j < ws(t) / g)
+            int t_lo, t_hi;
+            if (!kvalid) {
+                t_lo = 1;
+                t_hi = 0;
+            } else if (G.core) {
+                t_lo = (key + 1) * p.g + p.w;
+                t_hi = p.T - 1;
+            } else {
+                t_lo = key;
+                t_hi = min((key / p.g + 1) * p.g + p.w - 1, p.T - 1);
+            }
             for (int i = 0; i < n_tiles; ++i, ++it) {
                 const int kh = i / (G.qb - G.qa), qt = G.qa + (i - kh * (G.qb - G.qa));
                 const int hq = G.h * p.r + kh;
-                // per-column data of this query tile: log-sum-exp, D, window
-                // start (or core count), staged in shared memory
-                float *cb = col + (it & 1) * 3 * 128;
+                // per-column (log-sum-exp, D) of this query tile, staged in
+                // shared memory (double-buffered by tile)
+                const uint32_t cb = col_s + (it & 1) * 128 * 8;
                 {
                     const int t = qt * 128 + row;
                     const int64_t qrow = (static_cast<int64_t>(G.b) * p.Hq + hq) * p.T + t;
                     const bool tv = t < p.T;
-                    const int wst = ws_of(t, p.g, p.w);
-                    cb[row] = tv ? p.lse[qrow] : 0.f;
-                    cb[128 + row] = tv ? p.Dv[qrow] : 0.f;
-                    // raw: the lowest key t sees; core: the number of groups
-                    // it sees; a query past the end sees nothing
-                    cb[256 + row] = __int_as_float(tv ? (G.core ? wst / p.g : wst) : (G.core ? 0 : 1 << 30));
+                    const float lv = tv ? p.lse[qrow] : 0.f, dv_ = tv ? p.Dv[qrow] : 0.f;
+                    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(cb + row * 8), "f"(lv),
+                                 "f"(dv_)
+                                 : "memory");
                 }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
+                // this key's visible columns of the tile
+                const int c_lo = max(t_lo - qt * 128, 0), c_hi = min(t_hi - qt * 128, 127);
                 if (!(ok = bw_warp_wait(&bars->s_full, it & 1, bars))) break;
                 tc_fence_after_sync();
 #pragma unroll
@@ -703,19 +719,18 @@ __global__ void __launch_bounds__(192, 1)
                     tmem_wait_ld_dep(ud);
 #pragma unroll
                     for (int e = 0; e < 32; e += 2) {
-                        float pv[2], dsv[2];
-#pragma unroll
-                        for (int x = 0; x < 2; ++x) {
-                            const int cc = c * 32 + e + x;
-                            const int t = qt * 128 + cc;
-                            const int lim = __float_as_int(cb[256 + cc]);
-                            const bool vis = kvalid && (G.core ? key < lim : (key >= lim && key <= t));
-                            const float pr = vis ? fast_exp2(__uint_as_float(us[e + x]) * p.scale_log2 - cb[cc]) : 0.f;
-                            pv[x] = pr;
-                            dsv[x] = pr * (__uint_as_float(ud[e + x]) - cb[128 + cc]);
-                        }
-                        pp[e / 2] = pack16(pv[0], pv[1], G.core);
-                        pd[e / 2] = pack16(dsv[0], dsv[1], G.core);
+                        const int cc = c * 32 + e;
+                        float4 ld;  // (lse, D) of columns cc and cc + 1
+                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                     : "=f"(ld.x), "=f"(ld.y), "=f"(ld.z), "=f"(ld.w)
+                                     : "r"(cb + cc * 8));
+                        const bool v0 = cc >= c_lo && cc <= c_hi;
+                        const bool v1 = cc + 1 >= c_lo && cc + 1 <= c_hi;
+                        const float p0 = v0 ? fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - ld.x) : 0.f;
+                        const float p1 = v1 ? fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - ld.z) : 0.f;
+                        pp[e / 2] = pack16(p0, p1, G.core);
+                        pd[e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - ld.y),
+                                           p1 * (__uint_as_float(ud[e + 1]) - ld.w), G.core);
                     }
                     // over columns this thread has already read
                     tmem_st16(tmem + lane_off + L::ST_COL + c * 16, pp);
