@@ -56,7 +56,8 @@ TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.md
 # of them do not describe this one
 PREFILL_SOURCES = ("long_context_sparse_cca_b200/csrc/prefill.cu",
                    "long_context_sparse_cca_b200/csrc/sm100.cuh",
-                   "long_context_sparse_cca_b200/csrc/common.cuh")
+                   "long_context_sparse_cca_b200/csrc/common.cuh",
+                   "long_context_sparse_cca_b200/csrc/tma_map.h")
 
 
 # ----------------------------------------------------------------- workload arithmetic

@@ -102,12 +102,25 @@ struct Geom {
     int n_local, n_core_tiles, n_tiles;
 };
 
+// HM: head-major item order (all blocks of a head before the next head).
+template <bool HM>
 __device__ __forceinline__ Geom geom(int item, const Params &p)
 {
     Geom G;
     const int bhq_count = p.B * p.Hq;
-    const int blk = p.n_blocks - 1 - item / bhq_count;
-    const int bhq = item - (item / bhq_count) * bhq_count;
+    // Latest blocks (most core tiles) first.  Across heads when the core
+    // rows of all heads fit in L2, so that concurrent items have equal
+    // costs; head by head when they do not, so that each head's core rows
+    // are read from DRAM once (measured on B200 at 128K context: 4.2 GB of
+    // DRAM reads instead of 15.6 GB, 4-5% faster; at 32K, 11% slower).
+    int blk, bhq;
+    if constexpr (HM) {
+        bhq = item / p.n_blocks;
+        blk = p.n_blocks - 1 - (item - bhq * p.n_blocks);
+    } else {
+        blk = p.n_blocks - 1 - item / bhq_count;
+        bhq = item - (item / bhq_count) * bhq_count;
+    }
     G.b = bhq / p.Hq;
     G.hq = bhq - G.b * p.Hq;
     G.h = G.hq / p.r;
@@ -219,7 +232,8 @@ __device__ __forceinline__ float row_max128(const float (&x)[128])
 // LSE: also write each row's log-sum-exp (log2 units: log2 of the sum of
 // 2^(logit / ln 2) over the row's keys), which the backward kernels need;
 // a separate instance, so that the inference kernel is unchanged.
-template <int D, bool LSE>
+// HM: item order (geom), a separate instance for the same reason.
+template <int D, bool LSE, bool HM>
 __global__ void __launch_bounds__(352, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tmQ,
                    const __grid_constant__ CUtensorMap tmK,
@@ -285,7 +299,7 @@ __global__ void __launch_bounds__(352, 1)
             uint32_t kc = 0, vc = 0, qc = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-                const Geom G = geom(item, p);
+                const Geom G = geom<HM>(item, p);
                 if (qc > 0 && !(ok = lane_wait(&bars->q_empty, (qc - 1) & 1, bars))) break;
                 mbar_arrive_expect_tx(&bars->q_full, 2 * C::TILE_BYTES);
                 for (int hh = 0; hh < 2; ++hh)
@@ -372,7 +386,7 @@ __global__ void __launch_bounds__(352, 1)
                 };
                 for (int item = blockIdx.x; ok && item < p.n_items;
                      item += gridDim.x, ++k) {
-                    const Geom G = geom(item, p);
+                    const Geom G = geom<HM>(item, p);
                     if (!(ok = lane_wait(&bars->q_full, k & 1, bars))) break;
                     for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
                         const bool core = tile_is_core(G, j);
@@ -418,7 +432,7 @@ __global__ void __launch_bounds__(352, 1)
                 };
                 for (int item = blockIdx.x; ok && item < p.n_items;
                      item += gridDim.x, ++k) {
-                    const Geom G = geom(item, p);
+                    const Geom G = geom<HM>(item, p);
                     for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
                         const bool core = tile_is_core(G, j);
                         const uint32_t sv = vc % C::VST;
@@ -455,7 +469,7 @@ __global__ void __launch_bounds__(352, 1)
         uint32_t it = 0;  // key tiles over all items
         bool ok = true;
         for (int item = blockIdx.x; ok && item < p.n_items; item += gridDim.x) {
-            const Geom G = geom(item, p);
+            const Geom G = geom<HM>(item, p);
             const bool core_block = G.n_core_tiles > 0;
             const int t0h = G.t0 + hh * 128;       // first row of this half
             const int t = t0h + row;
@@ -656,11 +670,16 @@ cudaError_t launch_d(const void *Q, const void *K, const void *V, const void *Kc
     p.O = O;
     p.o_f32 = o_f32 ? 1 : 0;
     p.lse = lse;
-    int dev = 0, sms = 148;
+    int dev = 0, sms = 148, l2 = 0;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cudaDeviceGetAttribute(&l2, cudaDevAttrL2CacheSize, dev);
     const int grid = p.n_items < sms ? p.n_items : sms;
-    auto kern = lse ? prefill_kernel<D, true> : prefill_kernel<D, false>;
+    // head-major when the core keys and values of all heads (fp16) exceed
+    // half the L2
+    const bool hm = 4.0 * static_cast<double>(B) * Hkv * m * D > 0.5 * static_cast<double>(l2);
+    auto kern = lse ? (hm ? prefill_kernel<D, true, true> : prefill_kernel<D, true, false>)
+                    : (hm ? prefill_kernel<D, false, true> : prefill_kernel<D, false, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM);
     if (e != cudaSuccess) return e;
