@@ -67,6 +67,8 @@ def _bind(path: str):
     L.cca_oracle_window_start.restype = l
     L.cca_oracle_pool.argtypes = [P, P, P, P, P, P, i, i, i, l, i, i]
     L.cca_oracle_pool.restype = i
+    L.cca_oracle_lca_pool.argtypes = [P, P, P, P, P, P, P, i, i, i, l, i, i, i]
+    L.cca_oracle_lca_pool.restype = i
     L.cca_oracle_attend_rows.argtypes = [P, P, P, P, P, i, i, i, l, i, i, i,
                                          P, l, P]
     L.cca_oracle_attend_rows.restype = i
@@ -128,6 +130,27 @@ class Oracle:
                                         _ptr(Vc), _ptr(A), B, Hq, Hkv, T, d,
                                         g), "pool")
         return (Kc, Vc, A) if want_weights else (Kc, Vc)
+
+    def lca_pool(self, Q, K, V, g: int, d_rope: int, want_weights: bool = False):
+        """Latent-condensed pooling (the LCA variant).  Q [B,Hq,T,d],
+        K/V [B,Hkv,T,d]; the last d_rope entries of a key row are its
+        positional part.
+
+        Returns (Kc, Vc) [B,Hkv,m,d], plus the weights [B,Hkv,m,g] and the
+        anchor index per group [B,Hkv,m] if asked.
+        """
+        Q, K, V = _f64(Q), _f64(K), _f64(V)
+        B, Hq, T, d = Q.shape
+        Hkv = K.shape[1]
+        m = T // g
+        Kc = np.empty((B, Hkv, m, d))
+        Vc = np.empty((B, Hkv, m, d))
+        A = np.empty((B, Hkv, m, g)) if want_weights else None
+        anchor = np.empty((B, Hkv, m), dtype=np.int64) if want_weights else None
+        _check(self.lib.cca_oracle_lca_pool(_ptr(Q), _ptr(K), _ptr(V), _ptr(Kc),
+                                            _ptr(Vc), _ptr(A), _ptr(anchor), B, Hq,
+                                            Hkv, T, d, g, int(d_rope)), "lca_pool")
+        return (Kc, Vc, A, anchor) if want_weights else (Kc, Vc)
 
     def attend_rows(self, Q, K, V, Kc, Vc, g: int, w: int,
                     rows: Optional[Sequence[int]] = None) -> np.ndarray:
@@ -247,6 +270,10 @@ def window_start(t: int, g: int, w: int) -> int:
 
 def pool(Q, K, V, g: int, want_weights: bool = False):
     return default().pool(Q, K, V, g, want_weights)
+
+
+def lca_pool(Q, K, V, g: int, d_rope: int, want_weights: bool = False):
+    return default().lca_pool(Q, K, V, g, d_rope, want_weights)
 
 
 def attend_rows(Q, K, V, Kc, Vc, g: int, w: int, rows=None):

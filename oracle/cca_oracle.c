@@ -148,6 +148,98 @@ int cca_oracle_pool(const double *Q, const double *K, const double *V,
 }
 
 /*
+ * Latent-condensed pooling, the LCA variant (page "Latent-Condensed
+ * Transformer for Efficient Long Context Modeling", section 2 方法论,
+ * 核心设计思想: 语义凝聚 and 位置锚定).  A later method by the same group:
+ * history is split into groups; inside a group every token gets an
+ * importance score from the dot product of the group's average query with
+ * its key; the content part of the group is condensed by weighted pooling
+ * with these scores, while the positional part of the key (the rotary key
+ * K_R of multi-head latent attention) is not mixed: the group keeps the
+ * positional key of its highest-scoring token, the anchor.
+ *
+ * Readings taken (the summary gives no formulas):
+ *   - the average query of group j is the mean of the group's own g query
+ *     rows, q_bar = (1/g) sum_i q_{jg+i}, per query head;
+ *   - scores q_bar . k_i / sqrt(d) over the full key, normalised with a
+ *     softmax over the group (the pooling of the earlier CCA method);
+ *     with grouped-query attention the weights are the mean of the r query
+ *     heads' softmax vectors, as for CCA;
+ *   - the key row's last d_rope entries are its positional part and the
+ *     rest its content part (in the latent form the content key and the
+ *     value are linear in the latent vector C_KV, so pooling C_KV equals
+ *     pooling them with the same weights); values are content only;
+ *   - the anchor is the token of largest weight, the first one on a tie;
+ *   - a trailing partial group gets no core token (as for CCA).
+ * Writes Kc, Vc [B, Hkv, m, d]; if A is not NULL the weights [B, Hkv, m, g];
+ * if anchor is not NULL the anchor index within each group [B, Hkv, m].
+ */
+int cca_oracle_lca_pool(const double *Q, const double *K, const double *V,
+                        double *Kc, double *Vc, double *A, long *anchor, int B,
+                        int Hq, int Hkv, long T, int d, int g, int d_rope)
+{
+    if (B < 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv || T < 0 || d <= 0 ||
+        g <= 0 || d_rope < 0 || d_rope > d)
+        return CCA_ORACLE_EINVAL;
+    const int r = Hq / Hkv;
+    const long m = T / g;
+    const int d_content = d - d_rope;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+
+#pragma omp parallel num_threads(cca_oracle_threads())
+    {
+        double *qbar = (double *)malloc(sizeof(double) * (size_t)d);
+        double *p = (double *)malloc(sizeof(double) * (size_t)g);
+        double *wgt = (double *)malloc(sizeof(double) * (size_t)g);
+#pragma omp for collapse(3) schedule(static)
+        for (int b = 0; b < B; ++b)
+            for (int h = 0; h < Hkv; ++h)
+                for (long j = 0; j < m; ++j) {
+                    const long first = j * g;
+                    const double *Kg = K + (((size_t)b * Hkv + h) * T + first) * d;
+                    const double *Vg = V + (((size_t)b * Hkv + h) * T + first) * d;
+                    for (int i = 0; i < g; ++i) wgt[i] = 0.0;
+                    for (int k = 0; k < r; ++k) {
+                        const double *Qg =
+                            Q + (((size_t)b * Hq + h * r + k) * T + first) * d;
+                        /* the group's average query for this head */
+                        for (int c = 0; c < d; ++c) {
+                            double acc = 0.0;
+                            for (int i = 0; i < g; ++i) acc += Qg[(size_t)i * d + c];
+                            qbar[c] = acc / g;
+                        }
+                        for (int i = 0; i < g; ++i)
+                            p[i] = dot(qbar, Kg + (size_t)i * d, d) * inv_sqrt_d;
+                        softmax_inplace(p, g);
+                        for (int i = 0; i < g; ++i) wgt[i] += p[i] / (double)r;
+                    }
+                    int best = 0;
+                    for (int i = 1; i < g; ++i)
+                        if (wgt[i] > wgt[best]) best = i;
+                    const size_t out = ((size_t)b * Hkv + h) * m + j;
+                    double *kc = Kc + out * d;
+                    double *vc = Vc + out * d;
+                    for (int c = 0; c < d; ++c) {
+                        double kacc = 0.0, vacc = 0.0;
+                        for (int i = 0; i < g; ++i) {
+                            kacc += wgt[i] * Kg[(size_t)i * d + c];
+                            vacc += wgt[i] * Vg[(size_t)i * d + c];
+                        }
+                        kc[c] = c < d_content ? kacc : Kg[(size_t)best * d + c];
+                        vc[c] = vacc;
+                    }
+                    if (A)
+                        for (int i = 0; i < g; ++i) A[out * g + i] = wgt[i];
+                    if (anchor) anchor[out] = best;
+                }
+        free(qbar);
+        free(p);
+        free(wgt);
+    }
+    return CCA_ORACLE_OK;
+}
+
+/*
  * One query row of the fused attention (write-up, section 全局-局部模块可微融合
  * "differentiable global-local fusion"): the keys and values of the two
  * modules are concatenated into one key matrix and one value matrix, and the

@@ -45,6 +45,14 @@ int cca_oracle_pool(const double *Q, const double *K, const double *V,
                     double *Kc, double *Vc, double *A, int B, int Hq, int Hkv,
                     long T, int d, int g);
 
+/* Latent-condensed pooling (the LCA variant): weights from the group's
+ * average query, content dims [0, d - d_rope) pooled, positional dims
+ * [d - d_rope, d) copied from the group's highest-weight token.  Writes Kc,
+ * Vc [B, Hkv, m, d]; A [B, Hkv, m, g] and anchor [B, Hkv, m] when not NULL. */
+int cca_oracle_lca_pool(const double *Q, const double *K, const double *V,
+                        double *Kc, double *Vc, double *A, long *anchor, int B,
+                        int Hq, int Hkv, long T, int d, int g, int d_rope);
+
 /* Fused core + local attention for the query rows listed in rows[0..nrows)
  * (every batch entry and query head).  Kc, Vc are [B, Hkv, m, d] with
  * m = floor(T / g).  Writes O [B, Hq, nrows, d]. */

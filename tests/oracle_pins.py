@@ -227,6 +227,168 @@ def pin_pool_then_project_equals_project_then_pool(orc):
 
 
 # ---------------------------------------------------------------------------
+# latent-condensed pooling, the LCA variant (page "Latent-Condensed
+# Transformer for Efficient Long Context Modeling", section 2 方法论:
+# 语义凝聚, 位置锚定)
+# ---------------------------------------------------------------------------
+
+def _lca_anchor_group():
+    """One group of four tokens, d = 4, one head.  Queries (8,0,0,0), 0, 0, 0
+    average to (2,0,0,0), so token i scores x_i * 2 / sqrt(4) = x_i for a
+    key whose first entry is x_i.  With x = (0, ln 2, ln 4, 0) the weights
+    are (1, 2, 4, 1) / 8 and token 2 is the anchor.  The last query is zero:
+    it would give equal weights."""
+    x = np.array([0.0, math.log(2.0), math.log(4.0), 0.0])
+    Q = np.zeros((1, 1, 4, 4))
+    Q[0, 0, 0, 0] = 8.0
+    K = np.zeros((1, 1, 4, 4))
+    K[0, 0, :, 0] = x
+    K[0, 0, :, 1] = (1.0, -1.0, 0.5, 2.0)
+    K[0, 0, :, 2] = (3.0, 5.0, -7.0, 11.0)
+    K[0, 0, :, 3] = (-0.25, 0.75, 1.25, 0.5)
+    V = np.arange(16.0).reshape(1, 1, 4, 4) - 6.0
+    a = np.array([1.0, 2.0, 4.0, 1.0]) / 8.0
+    return Q, K, V, a
+
+
+def pin_lca_average_query_closed_form(orc):
+    """Weights from the group's average query (not its last query, not the
+    sum of its queries): (1, 2, 4, 1) / 8 for the group above."""
+    Q, K, V, a = _lca_anchor_group()
+    Kc, Vc, A, anchor = orc.lca_pool(Q, K, V, 4, 0, want_weights=True)
+    np.testing.assert_allclose(A[0, 0, 0], a, rtol=1e-14)
+    assert anchor[0, 0, 0] == 2
+    np.testing.assert_allclose(Kc[0, 0, 0], a @ K[0, 0], rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(Vc[0, 0, 0], a @ V[0, 0], rtol=1e-13, atol=1e-15)
+
+
+def pin_lca_anchor_keeps_positional_part(orc):
+    """d_rope = 2: the last two entries of the core key are the anchor's
+    own, (-7, 1.25) of token 2, copied, not pooled; the first two are
+    pooled; the value is pooled in full."""
+    Q, K, V, a = _lca_anchor_group()
+    Kc, Vc = orc.lca_pool(Q, K, V, 4, 2)
+    np.testing.assert_array_equal(Kc[0, 0, 0, 2:], [-7.0, 1.25])
+    np.testing.assert_allclose(Kc[0, 0, 0, :2], (a @ K[0, 0])[:2], rtol=1e-13)
+    np.testing.assert_allclose(Vc[0, 0, 0], a @ V[0, 0], rtol=1e-13, atol=1e-15)
+
+
+def pin_lca_all_positional_is_selection(orc):
+    """d_rope = d: the core key is the anchor's key row itself."""
+    Q, K, V, a = _lca_anchor_group()
+    Kc, Vc = orc.lca_pool(Q, K, V, 4, 4)
+    np.testing.assert_array_equal(Kc[0, 0, 0], K[0, 0, 2])
+    np.testing.assert_allclose(Vc[0, 0, 0], a @ V[0, 0], rtol=1e-13, atol=1e-15)
+
+
+def pin_lca_only_the_query_mean_matters(orc):
+    """Replacing a group's queries by others with the same mean changes
+    nothing; changing the mean changes the result."""
+    r = _rng(21)
+    B, H, T, d, g = 2, 2, 24, 8, 4
+    Q = r.standard_normal((B, H, T, d))
+    K = r.standard_normal((B, H, T, d))
+    V = r.standard_normal((B, H, T, d))
+    Kc, Vc = orc.lca_pool(Q, K, V, g, 4)
+    noise = r.standard_normal((B, H, T // g, g, d)) * 3
+    noise -= noise.mean(axis=3, keepdims=True)
+    Q2 = Q + noise.reshape(B, H, T, d)
+    Kc2, Vc2 = orc.lca_pool(Q2, K, V, g, 4)
+    np.testing.assert_allclose(Kc2, Kc, atol=1e-12)
+    np.testing.assert_allclose(Vc2, Vc, atol=1e-12)
+    Q3 = Q.copy()
+    Q3[:, :, g - 1::g] += r.standard_normal(Q3[:, :, g - 1::g].shape) * 3
+    _, Vc3 = orc.lca_pool(Q3, K, V, g, 4)
+    assert np.all(np.abs(Vc3 - Vc).max(-1) > 1e-6)
+
+
+def pin_lca_gqa_mean_of_head_softmaxes(orc):
+    """Two query heads on one key/value head, g = 2, d = 2.  Head 0's
+    queries average to (L sqrt2, 0), head 1's to (-L sqrt2, 0); with
+    k0 = (1, 0), k1 = 0 the heads' softmaxes are (e^L, 1)/(e^L + 1) and
+    (e^-L, 1)/(e^-L + 1), and the weights are their mean."""
+    L = 2.0
+    c = L * math.sqrt(2.0)
+    Q = np.zeros((1, 2, 2, 2))
+    Q[0, 0, 0] = (2 * c + 1.0, 3.0)
+    Q[0, 0, 1] = (-1.0, -3.0)
+    Q[0, 1, 0] = (-2 * c, 0.5)
+    Q[0, 1, 1] = (0.0, -0.5)
+    K = np.zeros((1, 1, 2, 2))
+    K[0, 0, 0] = (1.0, 0.0)
+    V = np.array([[[[1.0, 0.0], [0.0, 1.0]]]])
+    e = math.exp(L)
+    a = (np.array([e, 1.0]) / (e + 1.0) + np.array([1.0 / e, 1.0]) / (1.0 / e + 1.0)) / 2
+    Kc, Vc, A, anchor = orc.lca_pool(Q, K, V, 2, 0, want_weights=True)
+    np.testing.assert_allclose(A[0, 0, 0], a, rtol=1e-14)
+    np.testing.assert_allclose(Vc[0, 0, 0], a, rtol=1e-14)
+    assert anchor[0, 0, 0] == (0 if a[0] > a[1] else 1)
+
+
+def pin_lca_permutation_within_group(orc):
+    """Permuting a group's tokens (query, key and value rows together)
+    leaves its core token unchanged: the average query and the weighted sums
+    do not depend on the order, and the anchor moves with its token."""
+    r = _rng(22)
+    B, Hq, Hkv, T, d, g = 1, 4, 2, 30, 8, 6
+    Q = r.standard_normal((B, Hq, T, d))
+    K = r.standard_normal((B, Hkv, T, d))
+    V = r.standard_normal((B, Hkv, T, d))
+    perm = np.concatenate([j * g + r.permutation(g) for j in range(T // g)])
+    Kc, Vc = orc.lca_pool(Q, K, V, g, 4)
+    Kc2, Vc2 = orc.lca_pool(Q[:, :, perm], K[:, :, perm], V[:, :, perm], g, 4)
+    np.testing.assert_allclose(Kc2, Kc, atol=1e-12)
+    np.testing.assert_allclose(Vc2, Vc, atol=1e-12)
+
+
+def pin_lca_tie_takes_first_token(orc):
+    """Identical keys give equal weights: the anchor is the first token and
+    the core key is that key."""
+    r = _rng(23)
+    Q = r.standard_normal((1, 1, 5, 8))
+    K = np.broadcast_to(r.standard_normal((1, 1, 1, 8)), (1, 1, 5, 8)).copy()
+    V = r.standard_normal((1, 1, 5, 8))
+    Kc, Vc, A, anchor = orc.lca_pool(Q, K, V, 5, 3, want_weights=True)
+    assert anchor[0, 0, 0] == 0
+    np.testing.assert_allclose(A[0, 0, 0], 0.2, rtol=1e-14)
+    np.testing.assert_allclose(Kc[0, 0, 0], K[0, 0, 0], atol=1e-14)
+    np.testing.assert_allclose(Vc[0, 0, 0], V[0, 0].mean(0), atol=1e-14)
+
+
+def pin_lca_one_query_per_group_is_cca(orc):
+    """If every query of a group equals the group's last query, the average
+    query is that query, and with no positional part the condensed token is
+    CCA's pooled token (the earlier method of the same group, section
+    全局感知池化 of the CCA write-up)."""
+    r = _rng(24)
+    B, Hq, Hkv, T, d, g = 2, 4, 2, 27, 8, 3
+    Q = r.standard_normal((B, Hq, T, d))
+    Ql = Q.reshape(B, Hq, T // g, g, d)[:, :, :, g - 1:g]
+    Qs = np.broadcast_to(Ql, (B, Hq, T // g, g, d)).reshape(B, Hq, T, d)
+    K = r.standard_normal((B, Hkv, T, d))
+    V = r.standard_normal((B, Hkv, T, d))
+    Kc, Vc = orc.lca_pool(Qs, K, V, g, 0)
+    Kc1, Vc1 = orc.pool(Qs, K, V, g)
+    np.testing.assert_allclose(Kc, Kc1, atol=1e-13)
+    np.testing.assert_allclose(Vc, Vc1, atol=1e-13)
+
+
+def pin_lca_trailing_partial_group(orc):
+    """Tokens after the last complete group get no core token and do not
+    change the complete groups' core tokens."""
+    r = _rng(25)
+    B, H, d, g = 1, 2, 8, 4
+    Q = r.standard_normal((B, H, 23, d))
+    K = r.standard_normal((B, H, 23, d))
+    V = r.standard_normal((B, H, 23, d))
+    Kc, Vc = orc.lca_pool(Q, K, V, g, 4)
+    Kc2, Vc2 = orc.lca_pool(Q[:, :, :20], K[:, :, :20], V[:, :, :20], g, 4)
+    assert Kc.shape == (B, H, 5, d)
+    np.testing.assert_array_equal(Kc, Kc2)
+    np.testing.assert_array_equal(Vc, Vc2)
+
+
+# ---------------------------------------------------------------------------
 # fused attention (sections 局部保留模块, 全局-局部模块可微融合)
 # ---------------------------------------------------------------------------
 

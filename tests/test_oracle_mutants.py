@@ -38,6 +38,21 @@ MUTANTS = [
      "double *kc = c->k_core + (kv * c->core_cap + (j > 0 ? j - 1 : 0)) * d;", 0),
     ("decode ring index off by one", "kp[nc + i] = c->k_tail + (kv * c->tail_cap +\n                                              p % c->tail_cap) * d;",
      "kp[nc + i] = c->k_tail + (kv * c->tail_cap +\n                                              (p + 1) % c->tail_cap) * d;", 0),
+    ("lca scored by last query", "qbar[c] = acc / g;", "qbar[c] = Qg[(size_t)(g - 1) * d + c];", 0),
+    ("lca sum of queries", "qbar[c] = acc / g;", "qbar[c] = acc;", 0),
+    ("lca scale 1/d", "const double inv_sqrt_d = 1.0 / sqrt((double)d);",
+     "const double inv_sqrt_d = 1.0 / (double)d;", 0),
+    ("lca heads summed", "wgt[i] += p[i] / (double)r;", "wgt[i] += p[i];", 0),
+    ("lca anchor argmin", "if (wgt[i] > wgt[best]) best = i;", "if (wgt[i] < wgt[best]) best = i;", 0),
+    ("lca anchor last on ties", "if (wgt[i] > wgt[best]) best = i;", "if (wgt[i] >= wgt[best]) best = i;", 0),
+    ("lca positional part pooled", "kc[c] = c < d_content ? kacc : Kg[(size_t)best * d + c];",
+     "kc[c] = kacc;", 0),
+    ("lca positional part at the front", "kc[c] = c < d_content ? kacc : Kg[(size_t)best * d + c];",
+     "kc[c] = c >= d_rope ? kacc : Kg[(size_t)best * d + c];", 0),
+    ("lca values from keys", "vacc += wgt[i] * Vg[(size_t)i * d + c];",
+     "vacc += wgt[i] * Kg[(size_t)i * d + c];", 0),
+    ("lca query rows of head 0 only", "Q + (((size_t)b * Hq + h * r + k) * T + first) * d;",
+     "Q + (((size_t)b * Hq + h * r) * T + first) * d;", 0),
     ("capacity check off by one", "if (t / g >= c->core_cap) return CCA_ORACLE_ECAPACITY;",
      "if (t / g > c->core_cap) return CCA_ORACLE_ECAPACITY;", 0),
 ]
