@@ -51,6 +51,10 @@ L2_BYTES = 126 * 2 ** 20
 # the other prefill workloads of the method's evaluation shapes, timed beside
 # the headline one
 EXTRA_PREFILL = (synth.PREFILL_32K.name, synth.GQA_16K.name)
+# LCA variant: positional entries per key row (the rotary part of a
+# latent-attention key is 64 of its 192 entries in DeepSeek-V2; half of a
+# 128-entry head here)
+LCA_D_ROPE = 64
 TRAFFIC_PROFILE = os.path.join(ROOT, "profiles", "prefill_kernel_dram_traffic.md")
 # the sources of the prefill kernel: DRAM counters taken on another version
 # of them do not describe this one
@@ -82,6 +86,28 @@ def pool_bytes(wl) -> float:
     m = wl.T // wl.g
     return 2.0 * (2 * wl.B * wl.Hkv * wl.T * wl.d + wl.B * wl.Hq * m * wl.d +
                   2 * wl.B * wl.Hkv * m * wl.d)
+
+
+def lca_pool_bytes(wl) -> float:
+    """Algorithmic bytes of the LCA condensation: read every query row (the
+    group averages), K and V; write Kc, Vc (2-byte elements)."""
+    m = wl.T // wl.g
+    return 2.0 * (wl.B * wl.Hq * wl.T * wl.d + 2 * wl.B * wl.Hkv * wl.T * wl.d +
+                  2 * wl.B * wl.Hkv * m * wl.d)
+
+
+def lca_entry(wl, t: dict, pk: dict, world: int) -> dict:
+    """The LCA variant on one workload: condensation against HBM, then the
+    shared fused attention on the condensed rows."""
+    gbs = lca_pool_bytes(wl) / (t["lca_pool_ms"] * 1e-3) / 1e9
+    tf = prefill_flops(wl) / (t["prefill_ms"] * 1e-3) / 1e12
+    return {"tokens_per_s": world * wl.B * wl.T / ((t["lca_pool_ms"] + t["prefill_ms"]) * 1e-3),
+            "lca_pool_ms": t["lca_pool_ms"], "lca_pool_gbs": gbs,
+            "lca_pool_frac": gbs / pk["hbm_gbs"], "lca_pool_bytes": lca_pool_bytes(wl),
+            "prefill_ms": t["prefill_ms"], "prefill_tflops": tf,
+            "prefill_frac_burst": tf / pk["bf16_tflops"], "d_rope": LCA_D_ROPE,
+            "what": "cca_lca_pool (average-query weights, positional anchor) + "
+                    "cca_attn_prefill on the condensed rows"}
 
 
 def prefill_bytes(wl) -> float:
@@ -425,6 +451,12 @@ def run_cuda(args, rank: int, world: int, local_rank: int) -> dict:
         extra["backward"] = time_backward(cca, synth.PREFILL_32K, args.steps, args.warmup,
                                           stream, torch)
 
+    # --- the LCA variant on the headline inputs: condensation, then the
+    # shared fused attention (overwrites Kc, Vc, O after the timed region)
+    if do_prefill and not args.no_extra:
+        extra["lca"] = time_lca(cca, Q, K, V, Kc, Vc, O, pw, args.steps, args.warmup, stream,
+                                torch)
+
     # one all-reduce of every timing, the same on all ranks (no e2e: -1)
     total_ms, mean_pool, mean_prefill, mean_decode, mean_e2e = max_over_ranks(
         [total_ms, float(np.mean(pool_ms)), float(np.mean(prefill_ms)),
@@ -476,6 +508,25 @@ def time_backward(cca, wl, steps: int, warmup: int, stream, torch) -> dict:
     del Q, K, V, dO, Kc, Vc, O, lse, dQ, dK, dV, ws
     torch.cuda.empty_cache()
     return out
+
+
+def time_lca(cca, Q, K, V, Kc, Vc, O, wl, steps: int, warmup: int, stream, torch) -> dict:
+    """Mean CUDA-event times (ms) of cca_lca_pool and of cca_attn_prefill on
+    its rows, on resident inputs of workload wl."""
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)]
+           for _ in range(warmup + steps)]
+    for e in evs:
+        e[0].record(stream)
+        cca.cca_lca_pool(Q, K, V, wl.g, LCA_D_ROPE, Kc, Vc)
+        e[1].record(stream)
+        cca.cca_attn_prefill(Q, K, V, Kc, Vc, wl.g, wl.w, O=O)
+        e[2].record(stream)
+    torch.cuda.synchronize()
+    st = cca.cca_device_status()
+    assert st == cca.CCA_OK, cca.status_string(st)
+    timed = evs[warmup:]
+    return {"lca_pool_ms": float(np.mean([e[0].elapsed_time(e[1]) for e in timed])),
+            "prefill_ms": float(np.mean([e[1].elapsed_time(e[2]) for e in timed]))}
 
 
 def time_prefill(cca, wl, steps: int, warmup: int, stream, torch) -> dict:
@@ -723,7 +774,10 @@ def main(argv=None) -> int:
                             "bytes": dbytes,
                             "launches": "cca_decode_step: one kernel per token (append, split-K attention, merge)"},
             **{f"prefill[{name}]": prefill_entry(synth.WORKLOADS[name], t, pk, world)
-               for name, t in r["extra"].items() if name != "backward"},
+               for name, t in r["extra"].items() if name not in ("backward", "lca")},
+            **({"lca[" + args.prefill_wl.name + "]": lca_entry(args.prefill_wl, r["extra"]["lca"],
+                                                              pk, world)}
+               if "lca" in r["extra"] else {}),
             **({"backward[" + synth.PREFILL_32K.name + "]": backward_entry(
                 synth.PREFILL_32K, r["extra"]["backward"], pk, world)}
                if "backward" in r["extra"] else {}),

@@ -305,6 +305,60 @@ cca_status cca_attn_decode_noalloc(const cca_cache *c, const void *q_t, void *o_
                                    cca_dtype o_dtype, cudaStream_t stream);
 
 /*
+ * The LCA variant (page "Latent-Condensed Transformer for Efficient Long
+ * Context Modeling", section 2 方法论, 核心设计思想): a later method by the
+ * authors of CCA that condenses each group differently and keeps the same
+ * core + local attention.  Per group of g tokens and key/value head:
+ *   - semantic condensation (语义凝聚): every query head's average query
+ *     over the group's own g query rows scores the group's keys,
+ *     q_bar . k / sqrt(d); softmax per query head, mean over the r query
+ *     heads of the key/value head; the weights pool the value and the
+ *     content part of the key (entries [0, d - d_rope));
+ *   - positional anchoring (位置锚定): the positional part of the key (the
+ *     last d_rope entries: the rotary key of latent attention) is not mixed
+ *     but copied from the group's highest-weight token (the first one on a
+ *     tie).
+ * d_rope: 0 <= d_rope <= d, a multiple of 8 (CCA_ERR_INVALID_ARG
+ * otherwise).  The condensed rows (fp16, range clamp as for cca_pool) feed
+ * cca_attn_prefill and cca_attn_decode unchanged: the local window and the
+ * single softmax over [core ; raw] (section 局部上下文保留 and 推理流程 of
+ * that page) are CCA's.
+ */
+
+/* Condensation of every complete group: arguments, layout and errors as
+ * cca_pool, plus d_rope.  Reads every query row (the group averages), not
+ * only each group's last. */
+cca_status cca_lca_pool(const void *Q, const void *K, const void *V, void *Kc, void *Vc, int B,
+                        int Hq, int Hkv, int64_t T, int d, int g, int d_rope,
+                        cudaStream_t stream);
+
+/*
+ * Decode cache for the LCA variant (推理流程 of that page: the cache keeps
+ * the condensed rows and the newest w tokens, and condenses each group as
+ * it completes).  q_sum [B, Hq, d] (fp32, device memory, 16-byte aligned,
+ * caller-owned) holds per query head the sum of the query rows of the open
+ * (incomplete) group: a completed group needs its average query, and a
+ * query row is not kept once its token is appended.
+ *
+ * cca_lca_cache_prefill: as cca_cache_prefill, with cca_lca_pool's
+ * condensation; sets q_sum to the sums of the trailing partial group's
+ * query rows (zero if T is a multiple of g) and c->len = T.
+ *
+ * cca_lca_cache_append: as cca_cache_append for token t = c->len (ring slot
+ * t % tail_cap); adds q_t to q_sum, or, if t completes group j = t / g,
+ * condenses group j from the ring with average queries (q_sum + q_t) / g
+ * into core slot j and zeroes q_sum.  c->len becomes t + 1.
+ * CCA_ERR_CAPACITY (nothing written) if t / g >= core_cap.
+ *
+ * The same q_sum and d_rope must serve every call on one cache.  Decode
+ * attention is cca_attn_decode on the same cache.
+ */
+cca_status cca_lca_cache_prefill(cca_cache *c, float *q_sum, const void *Q, const void *K,
+                                 const void *V, int64_t T, int d_rope, cudaStream_t stream);
+cca_status cca_lca_cache_append(cca_cache *c, float *q_sum, const void *q_t, const void *k_t,
+                                const void *v_t, int d_rope, cudaStream_t stream);
+
+/*
  * Synchronise `stream`, then report CCA_ERR_CUDA if a CUDA error is
  * pending, CCA_ERR_TIMEOUT if any kernel of this library recorded a
  * timed-out wait since the last call, CCA_ERR_CAPACITY if a per-row call

@@ -46,7 +46,8 @@ EXPORTS = ("cca_pool", "cca_attn_prefill", "cca_cache_prefill",
            "cca_device_status", "cca_status_string", "cca_version", "cca_last_error",
            "cca_attn_decode_noalloc", "cca_selftest_wait_timeout",
            "cca_cache_append_rows", "cca_attn_decode_rows", "cca_decode_step",
-           "cca_attn_prefill_lse", "cca_attn_backward", "cca_attn_backward_workspace_bytes")
+           "cca_attn_prefill_lse", "cca_attn_backward", "cca_attn_backward_workspace_bytes",
+           "cca_lca_pool", "cca_lca_cache_prefill", "cca_lca_cache_append")
 
 
 class CCAError(RuntimeError):
@@ -92,6 +93,12 @@ def lib():
     L.cca_attn_backward.argtypes = [P, P, P, P, P, P, i, P, P, P, P, P, i, i, i, i64, i, i, i,
                                     P, ctypes.c_size_t, P]
     L.cca_attn_backward.restype = st
+    L.cca_lca_pool.argtypes = [P, P, P, P, P, i, i, i, i64, i, i, i, P]
+    L.cca_lca_pool.restype = i
+    L.cca_lca_cache_prefill.argtypes = [CP, P, P, P, P, i64, i, P]
+    L.cca_lca_cache_prefill.restype = i
+    L.cca_lca_cache_append.argtypes = [CP, P, P, P, P, i, P]
+    L.cca_lca_cache_append.restype = i
     L.cca_cache_prefill.argtypes = [CP, P, P, P, i64, P]
     L.cca_cache_prefill.restype = st
     L.cca_cache_append.argtypes = [CP, P, P, P, P]
@@ -364,6 +371,62 @@ def cca_cache_append(cache: Cache, q_t, k_t, v_t, stream=None) -> None:
     _check(lib().cca_cache_append(ctypes.byref(cache.struct), _dev(q_t, "q_t"),
                                   _dev(k_t, "k_t"), _dev(v_t, "v_t"),
                                   _stream(stream)), "cca_cache_append")
+
+
+# ---- the LCA variant: latent-condensed pooling with a positional anchor
+
+def cca_lca_pool(Q, K, V, g: int, d_rope: int, Kc=None, Vc=None, stream=None):
+    """LCA condensation: Q [B,Hq,T,d], K/V [B,Hkv,T,d] (bf16, CUDA); the last
+    d_rope entries of a key row are its positional part.
+
+    Returns (Kc, Vc) [B, Hkv, T // g, d] fp16, for cca_attn_prefill.
+    """
+    torch = _torch()
+    B, Hq, T, d = Q.shape
+    Hkv = K.shape[1]
+    m = T // g
+    if Kc is None:
+        Kc = torch.empty((B, Hkv, m, d), dtype=torch.float16, device=Q.device)
+    if Vc is None:
+        Vc = torch.empty((B, Hkv, m, d), dtype=torch.float16, device=Q.device)
+    if tuple(K.shape) != (B, Hkv, T, d) or tuple(V.shape) != (B, Hkv, T, d):
+        raise ValueError("K and V must be [B, Hkv, T, d]")
+    if tuple(Kc.shape) != (B, Hkv, m, d) or tuple(Vc.shape) != (B, Hkv, m, d):
+        raise ValueError("Kc and Vc must be [B, Hkv, T // g, d]")
+    _check(lib().cca_lca_pool(_dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"),
+                              _dev(Kc, "Kc", torch.float16), _dev(Vc, "Vc", torch.float16),
+                              B, Hq, Hkv, T, d, int(g), int(d_rope), _stream(stream)),
+           "cca_lca_pool")
+    return Kc, Vc
+
+
+def lca_query_sums(cache: Cache):
+    """A zeroed q_sum [B, Hq, d] fp32 buffer for the LCA cache calls."""
+    torch = _torch()
+    return torch.zeros((cache.B, cache.Hq, cache.d), dtype=torch.float32, device="cuda")
+
+
+def _qsum(cache: Cache, q_sum):
+    torch = _torch()
+    if tuple(q_sum.shape) != (cache.B, cache.Hq, cache.d):
+        raise ValueError("q_sum must be [B, Hq, d]")
+    return _dev(q_sum, "q_sum", torch.float32)
+
+
+def cca_lca_cache_prefill(cache: Cache, q_sum, Q, K, V, d_rope: int, stream=None) -> None:
+    """Fill ``cache`` from a prefix with LCA condensation; sets q_sum to the
+    open group's query sums."""
+    T = Q.shape[2]
+    _check(lib().cca_lca_cache_prefill(ctypes.byref(cache.struct), _qsum(cache, q_sum),
+                                       _dev(Q, "Q"), _dev(K, "K"), _dev(V, "V"), T,
+                                       int(d_rope), _stream(stream)), "cca_lca_cache_prefill")
+
+
+def cca_lca_cache_append(cache: Cache, q_sum, q_t, k_t, v_t, d_rope: int, stream=None) -> None:
+    """Append one token with LCA condensation of the group it completes."""
+    _check(lib().cca_lca_cache_append(ctypes.byref(cache.struct), _qsum(cache, q_sum),
+                                      _dev(q_t, "q_t"), _dev(k_t, "k_t"), _dev(v_t, "v_t"),
+                                      int(d_rope), _stream(stream)), "cca_lca_cache_append")
 
 
 def cca_decode_workspace_bytes(cache: Cache) -> int:

@@ -233,6 +233,80 @@ cca_status cca_cache_append(cca_cache *c, const void *q_t, const void *k_t,
     return CCA_OK;
 }
 
+// ---- the LCA variant -------------------------------------------------------
+
+cca_status cca_lca_pool(const void *Q, const void *K, const void *V, void *Kc, void *Vc, int B,
+                        int Hq, int Hkv, int64_t T, int d, int g, int d_rope,
+                        cudaStream_t stream)
+{
+    const cca_status s = shape_status(B, Hq, Hkv, T, d, g, 0);
+    if (s != CCA_OK) return s;
+    if (d_rope < 0 || d_rope > d || d_rope % 8 != 0) return CCA_ERR_INVALID_ARG;
+    const int64_t m = T / g;
+    const bool any = m > 0;
+    if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(Kc, any) ||
+        !ptr_ok(Vc, any))
+        return CCA_ERR_INVALID_ARG;
+    if (!any) return CCA_OK;
+    const size_t in_q = size_t(B) * Hq * T * d * 2, in_kv = size_t(B) * Hkv * T * d * 2;
+    const size_t out = size_t(B) * Hkv * m * d * 2;
+    if (overlap(Kc, out, Q, in_q) || overlap(Kc, out, K, in_kv) ||
+        overlap(Kc, out, V, in_kv) || overlap(Vc, out, Q, in_q) ||
+        overlap(Vc, out, K, in_kv) || overlap(Vc, out, V, in_kv) ||
+        overlap(Kc, out, Vc, out))
+        return CCA_ERR_INVALID_ARG;
+    return from_cuda(
+        cca::launch_lca_pool(Q, K, V, Kc, Vc, B, Hq, Hkv, T, d, g, d_rope, m, stream));
+}
+
+cca_status cca_lca_cache_prefill(cca_cache *c, float *q_sum, const void *Q, const void *K,
+                                 const void *V, int64_t T, int d_rope, cudaStream_t stream)
+{
+    cca_status s = cache_status(c);
+    if (s != CCA_OK) return s;
+    if (T < 0 || T > kMaxT) return CCA_ERR_INVALID_ARG;
+    if (d_rope < 0 || d_rope > c->d || d_rope % 8 != 0) return CCA_ERR_INVALID_ARG;
+    const bool any = T > 0;
+    if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(q_sum, true))
+        return CCA_ERR_INVALID_ARG;
+    if (any && (T - 1) / c->g >= c->core_cap) return CCA_ERR_CAPACITY;
+    const int64_t m = T / c->g;
+    cudaError_t e = cudaSuccess;
+    if (m > 0)
+        e = cca::launch_lca_pool(Q, K, V, c->k_core, c->v_core, c->B, c->Hq, c->Hkv, T, c->d,
+                                 c->g, d_rope, c->core_cap, stream);
+    if (e == cudaSuccess && any) {
+        const int64_t p0 = T > c->tail_cap ? T - c->tail_cap : 0;
+        e = cca::launch_tail_fill(K, V, c->k_tail, c->v_tail, c->B, c->Hkv, T, c->d, p0,
+                                  c->tail_cap, stream);
+    }
+    if (e == cudaSuccess)
+        e = cca::launch_lca_qsum_fill(Q, q_sum, c->B, c->Hq, c->d, T, m * c->g, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    c->len = T;
+    return CCA_OK;
+}
+
+cca_status cca_lca_cache_append(cca_cache *c, float *q_sum, const void *q_t, const void *k_t,
+                                const void *v_t, int d_rope, cudaStream_t stream)
+{
+    const cca_status s = cache_status(c);
+    if (s != CCA_OK) return s;
+    if (d_rope < 0 || d_rope > c->d || d_rope % 8 != 0) return CCA_ERR_INVALID_ARG;
+    if (!ptr_ok(q_t, true) || !ptr_ok(k_t, true) || !ptr_ok(v_t, true) ||
+        !ptr_ok(q_sum, true))
+        return CCA_ERR_INVALID_ARG;
+    const int64_t t = c->len;
+    if (t >= kMaxT || t / c->g >= c->core_cap) return CCA_ERR_CAPACITY;
+    const cudaError_t e = cca::launch_lca_append(q_t, k_t, v_t, q_sum, c->k_core, c->v_core,
+                                                 c->k_tail, c->v_tail, c->B, c->Hq, c->Hkv,
+                                                 c->d, c->g, d_rope, c->core_cap, c->tail_cap,
+                                                 t, stream);
+    if (e != cudaSuccess) return from_cuda(e);
+    c->len = t + 1;
+    return CCA_OK;
+}
+
 size_t cca_decode_workspace_bytes(const cca_cache *c)
 {
     if (cache_status(c) != CCA_OK) return 0;
@@ -330,15 +404,16 @@ cca_status cca_device_status(cudaStream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(stream);
     if (e != cudaSuccess) return from_cuda(e);
-    unsigned int a = 0, b = 0, c = 0, d = 0, f = 0, h = 0;
+    unsigned int a = 0, b = 0, c = 0, d = 0, f = 0, h = 0, l = 0;
     if ((e = cca::prefill_status_read_clear(&a)) != cudaSuccess ||
         (e = cca::pool_status_read_clear(&b)) != cudaSuccess ||
         (e = cca::append_status_read_clear(&c)) != cudaSuccess ||
         (e = cca::selftest_status_read_clear(&d)) != cudaSuccess ||
         (e = cca::decode_status_read_clear(&f)) != cudaSuccess ||
-        (e = cca::backward_status_read_clear(&h)) != cudaSuccess)
+        (e = cca::backward_status_read_clear(&h)) != cudaSuccess ||
+        (e = cca::lca_status_read_clear(&l)) != cudaSuccess)
         return from_cuda(e);
-    const unsigned int st = a | b | c | d | f | h;
+    const unsigned int st = a | b | c | d | f | h | l;
     if (st & cca::kStatusTimeout) return CCA_ERR_TIMEOUT;
     if (st & cca::kStatusCapacity) return CCA_ERR_CAPACITY;
     if (st & cca::kStatusRange) return CCA_ERR_RANGE;

@@ -79,6 +79,21 @@ cudaError_t launch_backward(const void *Q, const void *K, const void *V, const v
                             cudaStream_t s);
 cudaError_t backward_status_read_clear(unsigned int *v);
 
+// The LCA variant.  Condensation of all complete groups of Q/K/V into
+// Kc/Vc [B, Hkv, out_rows, d] (fp16; rows 0..floor(T/g)-1 written).
+cudaError_t launch_lca_pool(const void *Q, const void *K, const void *V, void *Kc, void *Vc,
+                            int B, int Hq, int Hkv, int64_t T, int d, int g, int d_rope,
+                            int64_t out_rows, cudaStream_t s);
+// Append token t with the running query sums q_sum [B, Hq, d] (fp32).
+cudaError_t launch_lca_append(const void *q_t, const void *k_t, const void *v_t, float *q_sum,
+                              void *k_core, void *v_core, void *k_tail, void *v_tail, int B,
+                              int Hq, int Hkv, int d, int g, int d_rope, int64_t core_cap,
+                              int64_t tail_cap, int64_t t, cudaStream_t s);
+// q_sum = sum of the query rows p0 .. T-1 of Q [B, Hq, T, d] (zero if none).
+cudaError_t launch_lca_qsum_fill(const void *Q, float *q_sum, int B, int Hq, int d, int64_t T,
+                                 int64_t p0, cudaStream_t s);
+cudaError_t lca_status_read_clear(unsigned int *v);
+
 // Device status words (bits kStatusTimeout, kStatusRange): read and clear.
 cudaError_t prefill_status_read_clear(unsigned int *v);
 cudaError_t pool_status_read_clear(unsigned int *v);

@@ -240,3 +240,43 @@ def test_rows_binding_checks_lens():
         cca.cca_cache_append_rows(c, torch.zeros(3, dtype=torch.int64), q, q, q)
     with pytest.raises(ValueError):
         cca.cca_attn_decode_rows(c, torch.zeros(2, dtype=torch.int32), q)
+
+
+def test_lca_argument_checks(L):
+    """The LCA calls refuse a bad d_rope, bad pointers and a full cache on
+    the host, before any launch; a refused append leaves the length."""
+    P = ctypes.c_void_p
+
+    def lpool(Q=FAKE, Kc=FAKE + 4096, d_rope=64, T=64, d=128):
+        return L.cca_lca_pool(P(Q), P(FAKE), P(FAKE), P(Kc), P(FAKE + 8192), 1, 2, 2, T, d,
+                              16, d_rope, None)
+
+    assert lpool(d_rope=4) == cca.CCA_ERR_INVALID_ARG   # not a multiple of 8
+    assert lpool(d_rope=-8) == cca.CCA_ERR_INVALID_ARG
+    assert lpool(d_rope=136) == cca.CCA_ERR_INVALID_ARG  # beyond d
+    assert lpool(Q=0) == cca.CCA_ERR_INVALID_ARG
+    assert lpool(Kc=FAKE) == cca.CCA_ERR_INVALID_ARG     # output overlaps an input
+    assert lpool(d=96) == cca.CCA_ERR_UNSUPPORTED
+    assert L.cca_lca_pool(None, None, None, None, None, 1, 2, 2, 15, 128, 16, 0,
+                          None) == cca.CCA_OK            # no complete group
+
+    QS = FAKE + (8 << 20)
+    c = _cache(length=10)
+    app = lambda qs=QS, q=FAKE, d_rope=64: L.cca_lca_cache_append(  # noqa: E731
+        ctypes.byref(c), P(qs), P(q), P(FAKE + 8192), P(FAKE + 16384), d_rope, None)
+    assert app(qs=0) == cca.CCA_ERR_INVALID_ARG
+    assert app(qs=QS + 4) == cca.CCA_ERR_INVALID_ARG     # misaligned sums
+    assert app(q=0) == cca.CCA_ERR_INVALID_ARG
+    assert app(d_rope=12) == cca.CCA_ERR_INVALID_ARG
+    assert c.len == 10
+    c = _cache(core_cap=2, length=32)  # token 32 belongs to group 2: no slot
+    assert app() == cca.CCA_ERR_CAPACITY
+    assert c.len == 32
+    c = _cache(core_cap=2)
+    assert L.cca_lca_cache_prefill(ctypes.byref(c), P(QS), P(FAKE), P(FAKE), P(FAKE), 33, 0,
+                                   None) == cca.CCA_ERR_CAPACITY
+    assert L.cca_lca_cache_prefill(ctypes.byref(c), None, P(FAKE), P(FAKE), P(FAKE), 20, 0,
+                                   None) == cca.CCA_ERR_INVALID_ARG
+    assert L.cca_lca_cache_prefill(ctypes.byref(c), P(QS), P(FAKE), P(FAKE), P(FAKE), 20, 130,
+                                   None) == cca.CCA_ERR_INVALID_ARG
+    assert c.len == 0
