@@ -173,9 +173,17 @@ __global__ void bw_prep_kernel(const uint16_t *__restrict__ dO, const void *__re
 // Work item: one 128-row query tile of one (batch, query head), latest tiles
 // first.  Key tiles as in the forward: local (raw keys ws(t0) .. last row,
 // bf16) then core (pooled keys 0 .. ws(last)/g - 1, fp16, against the fp16
-// copies of Q and dO, reloaded at the switch).  Warps 0-3: one query row per
-// thread; warp 4: TMA producer; warp 5: MMA issuer (one thread).
+// copies of Q and dO, reloaded at the switch).  Warps 0-7: the element-wise
+// dS step, thread (w % 4) * 32 + lane owning one query row and warps w < 4 /
+// w >= 4 its key columns [0, 64) / [64, 128) (a row needs no reduction);
+// warp 8: TMA producer; warp 9: MMA issuer (one thread).  The issuer runs
+// one tile ahead: S and dP of tile n+1 are issued once the dS warps have
+// copied tile n's into registers, before dQ += dS K of tile n, so the tensor
+// cores work while the dS step runs.
 // TMEM: S [0,128), dP [128,256), dS [256,320) (16-bit pairs), dQ [320, +D).
+constexpr int kDqSoftWarps = 8;
+constexpr int kDqTmaWarp = 8, kDqMmaWarp = 9;
+constexpr int kDqThreads = 320;
 template <int D>
 struct BqLayout {
     using T = Bt<D>;
@@ -211,7 +219,7 @@ __device__ __forceinline__ QGeom q_geom(int item, const BwParams &p)
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kDqThreads, 1)
     bw_dq_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                  const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
                  const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -242,16 +250,16 @@ __global__ void __launch_bounds__(192, 1)
             mbar_init(&bars->v_empty[s], 1);
         }
         mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->s_free, 4);
-        mbar_init(&bars->p_full, 4);
+        mbar_init(&bars->s_free, kDqSoftWarps);
+        mbar_init(&bars->p_full, kDqSoftWarps);
         mbar_init(&bars->mm_done, 1);
-        mbar_init(&bars->acc_empty, 4);
+        mbar_init(&bars->acc_empty, kDqSoftWarps);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         bars->never = 0;
         mbar_fence_init();
     }
-    if (warp == 4) {
+    if (warp == kDqTmaWarp) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
@@ -260,7 +268,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
+    if (warp == kDqTmaWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t kc = 0, vc = 0, qc = 0;
@@ -315,7 +323,7 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (qc > 0) wait_bounded(&bars->q_full[0], (qc - 1) & 1, never, kBwWaitNs);
         }
-    } else if (warp == 5) {
+    } else if (warp == kDqMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
             constexpr uint32_t id_s_bf = idesc_f32acc(128, 128, true, false, false);
@@ -328,43 +336,80 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t dkm = smem_desc_sw128(smem_addr(sK), T::BOX_BYTES, 1024);
             const uint64_t dv = smem_desc_sw128(smem_addr(sV), 16, 1024);
             constexpr uint32_t kTile16 = T::TILE_BYTES >> 4;
-            uint32_t kc = 0, vc = 0, qc = 0, it = 0;
-            int k = 0;
-            bool ok = true;
-            for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
-                const QGeom G = q_geom(item, p);
-                if (!(ok = bw_lane_wait(&bars->q_full[0], qc & 1, bars))) break;
-                ++qc;
-                for (int j = 0; ok && j < G.n_tiles; ++j, ++it) {
-                    const bool core = j >= G.n_local;
-                    if (core && j == G.n_local) {
-                        // the bf16 query tiles are read: swap in the fp16 copies
-                        mma_commit(&bars->q_empty[0]);
-                        if (!(ok = bw_lane_wait(&bars->q_full[0], qc & 1, bars))) break;
-                        ++qc;
-                    }
-                    const uint32_t s = kc % L::KST, sv = vc % L::VST;
-                    if (!(ok = bw_lane_wait(&bars->k_full[s], (kc / L::KST) & 1, bars))) break;
-                    if (!(ok = bw_lane_wait(&bars->v_full[sv], (vc / L::VST) & 1, bars))) break;
-                    if (it > 0 && !(ok = bw_lane_wait(&bars->s_free, (it - 1) & 1, bars))) break;
-                    tc_fence_after_sync();
-                    mma_kk<D>(tmem + L::S_COL, dq, dk + s * kTile16, core ? id_s_h : id_s_bf);
-                    mma_kk<D>(tmem + L::DP_COL, dO, dv + sv * kTile16, core ? id_s_h : id_s_bf);
-                    mma_commit(&bars->s_full);
-                    mma_commit(&bars->v_empty[sv]);
-                    ++vc;
-                    if (!(ok = bw_lane_wait(&bars->p_full, it & 1, bars))) break;
-                    if (j == 0 && k > 0 && !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
-                        break;
-                    tc_fence_after_sync();
-                    mma_tm(tmem + L::DQ_COL, tmem + L::DS_COL, dkm + s * kTile16,
-                           core ? id_q_h : id_q_bf, j == 0);
-                    mma_commit(&bars->mm_done);
-                    mma_commit(&bars->k_empty[s]);
-                    ++kc;
+            // Tiles are numbered n = 0, 1, ... over this CTA's items in
+            // order; tile n uses K stage n % KST and V stage n % VST.  A(n)
+            // issues S, dP of tile n; B(n) issues dQ += dS K of tile n.
+            // Order: A(0), A(1), B(0), A(2), B(1), ...
+            struct Cursor {
+                int item, k, j;  // item index, its ordinal in this CTA, tile within it
+                QGeom G;
+                bool live;
+            };
+            auto start = [&](Cursor &c) {
+                c.item = blockIdx.x;
+                c.k = 0;
+                c.j = 0;
+                c.live = c.item < n_items;
+                if (c.live) c.G = q_geom(c.item, p);
+            };
+            auto advance = [&](Cursor &c) {
+                if (++c.j == c.G.n_tiles) {
+                    c.item += gridDim.x;
+                    ++c.k;
+                    c.j = 0;
+                    c.live = c.item < n_items;
+                    if (c.live) c.G = q_geom(c.item, p);
                 }
-                if (!ok) break;
-                mma_commit(&bars->q_empty[0]);
+            };
+            Cursor ca, cb;
+            start(ca);
+            start(cb);
+            uint32_t na = 0, nb = 0, qc = 0;
+            auto issue_a = [&]() -> bool {
+                const bool core = ca.j >= ca.G.n_local;
+                if (ca.j == 0 || (core && ca.j == ca.G.n_local)) {
+                    // this item's query tiles (bf16), or their fp16 copies
+                    if (!bw_lane_wait(&bars->q_full[0], qc & 1, bars)) return false;
+                    ++qc;
+                }
+                const uint32_t s = na % L::KST, sv = na % L::VST;
+                if (!bw_lane_wait(&bars->k_full[s], (na / L::KST) & 1, bars)) return false;
+                if (!bw_lane_wait(&bars->v_full[sv], (na / L::VST) & 1, bars)) return false;
+                if (na > 0 && !bw_lane_wait(&bars->s_free, (na - 1) & 1, bars)) return false;
+                tc_fence_after_sync();
+                mma_kk<D>(tmem + L::S_COL, dq, dk + s * kTile16, core ? id_s_h : id_s_bf);
+                mma_kk<D>(tmem + L::DP_COL, dO, dv + sv * kTile16, core ? id_s_h : id_s_bf);
+                mma_commit(&bars->s_full);
+                mma_commit(&bars->v_empty[sv]);
+                // the query tiles in shared memory are read for the last
+                // time: before the switch to the fp16 copies, and at the
+                // item's last tile
+                if (ca.j + 1 == ca.G.n_tiles || (!core && ca.j + 1 == ca.G.n_local))
+                    mma_commit(&bars->q_empty[0]);
+                ++na;
+                advance(ca);
+                return true;
+            };
+            auto issue_b = [&]() -> bool {
+                const bool core = cb.j >= cb.G.n_local;
+                if (!bw_lane_wait(&bars->p_full, nb & 1, bars)) return false;
+                if (cb.j == 0 && cb.k > 0 &&
+                    !bw_lane_wait(&bars->acc_empty, (cb.k - 1) & 1, bars))
+                    return false;
+                tc_fence_after_sync();
+                const uint32_t s = nb % L::KST;
+                mma_tm(tmem + L::DQ_COL, tmem + L::DS_COL, dkm + s * kTile16,
+                       core ? id_q_h : id_q_bf, cb.j == 0);
+                mma_commit(&bars->mm_done);
+                mma_commit(&bars->k_empty[s]);
+                ++nb;
+                advance(cb);
+                return true;
+            };
+            bool ok = !ca.live || issue_a();
+            while (ok && nb < na) {
+                if (ca.live && !(ok = issue_a())) break;
+                ok = issue_b();
             }
             mma_commit(&bars->drain);
             wait_bounded(&bars->drain, 0, &bars->never, kBwWaitNs);
@@ -372,6 +417,7 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         // ------------------------------------------------ dS warps
         const int row = threadIdx.x & 127;
+        const int half = warp >> 2;  // key columns [64 half, 64 half + 64)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         uint32_t it = 0;
         bool ok = true;
@@ -390,9 +436,10 @@ __global__ void __launch_bounds__(192, 1)
                 const bool core = j >= G.n_local;
                 const int key0 = core ? (j - G.n_local) * 128 : G.ws_lo + j * 128;
                 const int lo = core ? 0 : ws_t, hi = core ? nc_t - 1 : t;
-                uint32_t pk[4][16];
+                uint32_t pk[2][16];
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
+                for (int cc = 0; cc < 2; ++cc) {
+                    const int c = 2 * half + cc;
                     uint32_t us[32], ud[32];
                     tmem_ld32(tmem + lane_off + L::S_COL + c * 32, us);
                     tmem_ld32(tmem + lane_off + L::DP_COL + c * 32, ud);
@@ -405,8 +452,8 @@ __global__ void __launch_bounds__(192, 1)
                         const bool v1 = valid && key + 1 >= lo && key + 1 <= hi;
                         const float p0 = v0 ? fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - lse) : 0.f;
                         const float p1 = v1 ? fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - lse) : 0.f;
-                        pk[c][e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - dd),
-                                              p1 * (__uint_as_float(ud[e + 1]) - dd), core);
+                        pk[cc][e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - dd),
+                                               p1 * (__uint_as_float(ud[e + 1]) - dd), core);
                     }
                 }
                 tc_fence_before_sync();
@@ -418,7 +465,8 @@ __global__ void __launch_bounds__(192, 1)
                     tc_fence_after_sync();
                 }
 #pragma unroll
-                for (int c = 0; c < 4; ++c) tmem_st16(tmem + lane_off + L::DS_COL + c * 16, pk[c]);
+                for (int cc = 0; cc < 2; ++cc)
+                    tmem_st16(tmem + lane_off + L::DS_COL + (2 * half + cc) * 16, pk[cc]);
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncwarp();
@@ -429,7 +477,8 @@ __global__ void __launch_bounds__(192, 1)
             if (!(ok = bw_warp_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
             tc_fence_after_sync();
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int cc = 0; cc < D / 64; ++cc) {
+                const int c = half * (D / 64) + cc;
                 uint32_t u[32];
                 tmem_ld32_wait(tmem + lane_off + L::DQ_COL + c * 32, u);
                 if (valid) {
@@ -449,7 +498,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == kDqTmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
@@ -985,7 +1034,8 @@ cudaError_t launch_bw(const void *Q, const void *K, const void *V, const void *K
         if ((e = cudaFuncSetAttribute(bw_dq_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       LQ::SMEM)) != cudaSuccess)
             return e;
-        bw_dq_kernel<D><<<grid, 192, LQ::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc, mVc, p);
+        bw_dq_kernel<D><<<grid, kDqThreads, LQ::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc, mVc,
+                                                            p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 3. dK, dV and dKc, dVc
