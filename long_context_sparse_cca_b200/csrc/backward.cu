@@ -23,6 +23,8 @@
 //      dK += dS^T Q; raw tiles store dK, dV; core tiles (whose query range
 //      is long, so it is cut into chunks) add into fp32 dKc, dVc;
 //   4. bw_pool_kernel: one warp per group, the pooling's chain rule.
+#include <type_traits>
+
 #include "common.cuh"
 #include "internal.h"
 #include "sm100.cuh"
@@ -71,6 +73,7 @@ struct BwBars {
     uint64_t v_full[4], v_empty[4];
     uint64_t kv_full, kv_empty;      // key-side tiles (dK/dV kernel)
     uint64_t s_full, s_free, p_full, mm_done, acc_empty, drain;
+    uint64_t hs_full[2], hp_full[2], hmm_done[2];  // per 64-query half (dK/dV kernel)
     uint32_t tmem_base;
     int abort, never;
 };
@@ -109,6 +112,16 @@ __device__ __forceinline__ void mma_kk(uint32_t d_tmem, uint64_t a0, uint64_t b0
     }
 }
 
+// 128 x D x 64 product: A (16-bit pairs, 32 columns) in TMEM, B MN-major in
+// shared memory (64 rows along K); accumulate unless `first`.
+__device__ __forceinline__ void mma_tm64(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                         uint32_t idesc, bool first)
+{
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+        mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc, (first && kk == 0) ? 0u : 1u);
+}
+
 // 128 x D x 128 product: A (16-bit pairs) in TMEM, B MN-major in shared
 // memory; accumulate unless `first`.
 __device__ __forceinline__ void mma_tm(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
@@ -117,6 +130,15 @@ __device__ __forceinline__ void mma_tm(uint32_t d_tmem, uint32_t a_tmem, uint64_
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
         mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc, (first && kk == 0) ? 0u : 1u);
+}
+
+// Four fp32 additions to global memory in one 16-byte reduction (p 16-byte
+// aligned); the order among concurrent adders is unspecified.
+__device__ __forceinline__ void red_add_v4(float *ptr, float a, float b, float c, float d)
+{
+    asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(ptr), "f"(a),
+                 "f"(b), "f"(c), "f"(d)
+                 : "memory");
 }
 
 __device__ __forceinline__ uint32_t pack16(float a, float b, bool f16)
@@ -437,24 +459,48 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 const int key0 = core ? (j - G.n_local) * 128 : G.ws_lo + j * 128;
                 const int lo = core ? 0 : ws_t, hi = core ? nc_t - 1 : t;
                 uint32_t pk[2][16];
+                // CORE: fp16 dS (core tiles) or bf16; MASK: test each key
+                // against [lo, hi], skipped when every key of this half is
+                // visible to every row of the warp
+                auto elementwise = [&](auto core_c, auto mask_c) {
+                    constexpr bool CORE = decltype(core_c)::value;
+                    constexpr bool MASK = decltype(mask_c)::value;
 #pragma unroll
-                for (int cc = 0; cc < 2; ++cc) {
-                    const int c = 2 * half + cc;
-                    uint32_t us[32], ud[32];
-                    tmem_ld32(tmem + lane_off + L::S_COL + c * 32, us);
-                    tmem_ld32(tmem + lane_off + L::DP_COL + c * 32, ud);
-                    tmem_wait_ld_dep(us);
-                    tmem_wait_ld_dep(ud);
+                    for (int cc = 0; cc < 2; ++cc) {
+                        const int c = 2 * half + cc;
+                        uint32_t us[32], ud[32];
+                        tmem_ld32(tmem + lane_off + L::S_COL + c * 32, us);
+                        tmem_ld32(tmem + lane_off + L::DP_COL + c * 32, ud);
+                        tmem_wait_ld_dep(us);
+                        tmem_wait_ld_dep(ud);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int key = key0 + c * 32 + e;
-                        const bool v0 = valid && key >= lo && key <= hi;
-                        const bool v1 = valid && key + 1 >= lo && key + 1 <= hi;
-                        const float p0 = v0 ? fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - lse) : 0.f;
-                        const float p1 = v1 ? fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - lse) : 0.f;
-                        pk[cc][e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - dd),
-                                               p1 * (__uint_as_float(ud[e + 1]) - dd), core);
+                        for (int e = 0; e < 32; e += 2) {
+                            const int key = key0 + c * 32 + e;
+                            float p0 = fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - lse);
+                            float p1 = fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - lse);
+                            if (MASK) {
+                                p0 = valid && key >= lo && key <= hi ? p0 : 0.f;
+                                p1 = valid && key + 1 >= lo && key + 1 <= hi ? p1 : 0.f;
+                            }
+                            const float d0 = p0 * (__uint_as_float(ud[e]) - dd);
+                            const float d1 = p1 * (__uint_as_float(ud[e + 1]) - dd);
+                            pk[cc][e / 2] = CORE ? pack_f16x2(d0, d1) : pack_bf16x2(d0, d1);
+                        }
                     }
+                };
+                const int k_first = key0 + 64 * half;
+                const bool full =
+                    __all_sync(0xffffffffu, valid && k_first >= lo && k_first + 63 <= hi);
+                if (core) {
+                    if (full)
+                        elementwise(std::true_type{}, std::false_type{});
+                    else
+                        elementwise(std::true_type{}, std::true_type{});
+                } else {
+                    if (full)
+                        elementwise(std::false_type{}, std::false_type{});
+                    else
+                        elementwise(std::false_type{}, std::true_type{});
                 }
                 tc_fence_before_sync();
                 __syncwarp();
@@ -511,9 +557,12 @@ __global__ void __launch_bounds__(kDqThreads, 1)
 // query range (every later query sees a core key) cut into chunks of
 // kCoreChunk tiles whose results are added into fp32 dKc, dVc; raw tiles
 // take every query tile that sees one of their keys and store dK, dV.
-// Warps 0-3: one key row per thread; warp 4: TMA producer; warp 5: issuer.
-// TMEM: S^T [0,128) then P^T over its first 64 columns; dP^T [128,256) then
-// dS^T over its first 64; dK [256, 256+D); dV [256+D, 256+2D).
+// Each (key tile, query tile) pair runs as two 64-query halves h, so that
+// the element-wise step of one half overlaps the MMAs of the other:
+// warps 4h .. 4h+3 take half h (one key row per thread); warp 8: TMA
+// producer; warp 9: issuer.  TMEM: S^T [0,128), half h in [64h, 64h+64),
+// then that half's P^T over its first 32 columns; dP^T [128,256) the same
+// way with dS^T; dK [256, 256+D); dV [256+D, 256+2D).
 template <int D>
 struct BkLayout {
     using T = Bt<D>;
@@ -526,6 +575,10 @@ struct BkLayout {
     static constexpr int SMEM = OFF_BAR + 512 + 1024;
     static constexpr uint32_t ST_COL = 0, DPT_COL = 128, DK_COL = 256, DV_COL = 256 + D;
 };
+
+constexpr int kDkvSoftWarps = 8;
+constexpr int kDkvTmaWarp = 8, kDkvMmaWarp = 9;
+constexpr int kDkvThreads = 320;
 
 struct KGeom {
     bool core;
@@ -577,7 +630,7 @@ __device__ __forceinline__ KGeom k_geom(int item, const BwParams &p)
 }
 
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(kDkvThreads, 1)
     bw_dkv_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmO,
                   const __grid_constant__ CUtensorMap tmQ16, const __grid_constant__ CUtensorMap tmO16,
                   const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
@@ -604,16 +657,18 @@ __global__ void __launch_bounds__(192, 1)
         }
         mbar_init(&bars->kv_full, 1);
         mbar_init(&bars->kv_empty, 1);
-        mbar_init(&bars->s_full, 1);
-        mbar_init(&bars->p_full, 4);
-        mbar_init(&bars->mm_done, 1);
-        mbar_init(&bars->acc_empty, 4);
+        for (int h = 0; h < 2; ++h) {
+            mbar_init(&bars->hs_full[h], 1);
+            mbar_init(&bars->hp_full[h], 4);
+            mbar_init(&bars->hmm_done[h], 1);
+        }
+        mbar_init(&bars->acc_empty, kDkvSoftWarps);
         mbar_init(&bars->drain, 1);
         bars->abort = 0;
         bars->never = 0;
         mbar_fence_init();
     }
-    if (warp == 4) {
+    if (warp == kDkvTmaWarp) {
         tmem_alloc(&bars->tmem_base, 512);
         tmem_relinquish();
     }
@@ -622,7 +677,7 @@ __global__ void __launch_bounds__(192, 1)
     tc_fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
 
-    if (warp == 4) {
+    if (warp == kDkvTmaWarp) {
         // ------------------------------------------------ TMA producer
         if (lane == 0) {
             uint32_t qc = 0, kvc = 0;
@@ -665,11 +720,11 @@ __global__ void __launch_bounds__(192, 1)
             }
             if (kvc > 0) wait_bounded(&bars->kv_full, (kvc - 1) & 1, never, kBwWaitNs);
         }
-    } else if (warp == 5) {
+    } else if (warp == kDkvMmaWarp) {
         // ------------------------------------------------ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t id_s_bf = idesc_f32acc(128, 128, true, false, false);
-            constexpr uint32_t id_s_h = idesc_f32acc(128, 128, false, false, false);
+            constexpr uint32_t id_s_bf = idesc_f32acc(128, 64, true, false, false);
+            constexpr uint32_t id_s_h = idesc_f32acc(128, 64, false, false, false);
             constexpr uint32_t id_a_bf = idesc_f32acc(128, D, true, false, true);
             constexpr uint32_t id_a_h = idesc_f32acc(128, D, false, false, true);
             const uint64_t dk = smem_desc_sw128(smem_addr(sK), 16, 1024);
@@ -679,6 +734,7 @@ __global__ void __launch_bounds__(192, 1)
             const uint64_t dO = smem_desc_sw128(smem_addr(sO), 16, 1024);
             const uint64_t dOm = smem_desc_sw128(smem_addr(sO), T::BOX_BYTES, 1024);
             constexpr uint32_t kTile16 = T::TILE_BYTES >> 4;
+            constexpr uint32_t kHalf16 = (64 * 128) >> 4;  // 64 rows of a swizzled box
             uint32_t qc = 0, it = 0, kvc = 0;
             int k = 0;
             bool ok = true;
@@ -691,19 +747,32 @@ __global__ void __launch_bounds__(192, 1)
                 for (int i = 0; ok && i < n_tiles; ++i, ++it) {
                     const uint32_t s = qc % L::QST;
                     if (!(ok = bw_lane_wait(&bars->q_full[s], (qc / L::QST) & 1, bars))) break;
-                    // the previous tile's dV, dK products have read P^T, dS^T
-                    if (it > 0 && !(ok = bw_lane_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
-                    tc_fence_after_sync();
-                    mma_kk<D>(tmem + L::ST_COL, dk, dq + s * kTile16, ids);
-                    mma_kk<D>(tmem + L::DPT_COL, dv, dO + s * kTile16, ids);
-                    mma_commit(&bars->s_full);
-                    if (!(ok = bw_lane_wait(&bars->p_full, it & 1, bars))) break;
-                    if (i == 0 && k > 0 && !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
-                        break;
-                    tc_fence_after_sync();
-                    mma_tm(tmem + L::DV_COL, tmem + L::ST_COL, dOm + s * kTile16, ida, i == 0);
-                    mma_tm(tmem + L::DK_COL, tmem + L::DPT_COL, dqm + s * kTile16, ida, i == 0);
-                    mma_commit(&bars->mm_done);
+                    // S^T, dP^T of both halves; half h waits until the
+                    // previous tile's dV, dK products have read its P^T, dS^T
+                    for (int h = 0; ok && h < 2; ++h) {
+                        if (it > 0 && !(ok = bw_lane_wait(&bars->hmm_done[h], (it - 1) & 1, bars)))
+                            break;
+                        tc_fence_after_sync();
+                        mma_kk<D>(tmem + L::ST_COL + 64 * h, dk, dq + s * kTile16 + h * kHalf16, ids);
+                        mma_kk<D>(tmem + L::DPT_COL + 64 * h, dv, dO + s * kTile16 + h * kHalf16,
+                                  ids);
+                        mma_commit(&bars->hs_full[h]);
+                    }
+                    // dV += P^T dO, dK += dS^T Q, half by half
+                    for (int h = 0; ok && h < 2; ++h) {
+                        if (!(ok = bw_lane_wait(&bars->hp_full[h], it & 1, bars))) break;
+                        if (h == 0 && i == 0 && k > 0 &&
+                            !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
+                            break;
+                        tc_fence_after_sync();
+                        const bool first = i == 0 && h == 0;
+                        mma_tm64(tmem + L::DV_COL, tmem + L::ST_COL + 64 * h,
+                                 dOm + s * kTile16 + h * 512, ida, first);
+                        mma_tm64(tmem + L::DK_COL, tmem + L::DPT_COL + 64 * h,
+                                 dqm + s * kTile16 + h * 512, ida, first);
+                        mma_commit(&bars->hmm_done[h]);
+                    }
+                    if (!ok) break;
                     mma_commit(&bars->q_empty[s]);
                     ++qc;
                 }
@@ -716,6 +785,7 @@ __global__ void __launch_bounds__(192, 1)
     } else {
         // ------------------------------------------------ P^T, dS^T warps
         const int row = threadIdx.x & 127;
+        const int half = warp >> 2;  // query columns [64 half, 64 half + 64)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         uint32_t it = 0;
         bool ok = true;
@@ -742,72 +812,104 @@ __global__ void __launch_bounds__(192, 1)
             for (int i = 0; i < n_tiles; ++i, ++it) {
                 const int kh = i / (G.qb - G.qa), qt = G.qa + (i - kh * (G.qb - G.qa));
                 const int hq = G.h * p.r + kh;
-                // per-column (log-sum-exp, D) of this query tile, staged in
-                // shared memory (double-buffered by tile)
+                // per-column (log-sum-exp, D) of this half's 64 query
+                // columns, staged in shared memory (double-buffered by tile)
                 const uint32_t cb = col_s + (it & 1) * 128 * 8;
-                {
-                    const int t = qt * 128 + row;
+                if (row < 64) {
+                    const int col = 64 * half + row;
+                    const int t = qt * 128 + col;
                     const int64_t qrow = (static_cast<int64_t>(G.b) * p.Hq + hq) * p.T + t;
                     const bool tv = t < p.T;
                     const float lv = tv ? p.lse[qrow] : 0.f, dv_ = tv ? p.Dv[qrow] : 0.f;
-                    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(cb + row * 8), "f"(lv),
+                    asm volatile("st.shared.v2.f32 [%0], {%1, %2};" ::"r"(cb + col * 8), "f"(lv),
                                  "f"(dv_)
                                  : "memory");
                 }
-                asm volatile("bar.sync 1, 128;" ::: "memory");
+                asm volatile("bar.sync %0, 128;" ::"r"(1 + half) : "memory");
                 // this key's visible columns of the tile
                 const int c_lo = max(t_lo - qt * 128, 0), c_hi = min(t_hi - qt * 128, 127);
-                if (!(ok = bw_warp_wait(&bars->s_full, it & 1, bars))) break;
+                if (!(ok = bw_warp_wait(&bars->hs_full[half], it & 1, bars))) break;
                 tc_fence_after_sync();
+                // CORE: fp16 P, dS (core tiles) or bf16; MASK: test each
+                // column against [c_lo, c_hi], skipped when every column of
+                // this half is visible to every key row of the warp
+                auto elementwise = [&](auto core_c, auto mask_c) {
+                    constexpr bool CORE = decltype(core_c)::value;
+                    constexpr bool MASK = decltype(mask_c)::value;
 #pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    uint32_t us[32], ud[32], pp[16], pd[16];
-                    tmem_ld32(tmem + lane_off + L::ST_COL + c * 32, us);
-                    tmem_ld32(tmem + lane_off + L::DPT_COL + c * 32, ud);
-                    tmem_wait_ld_dep(us);
-                    tmem_wait_ld_dep(ud);
+                    for (int h2 = 0; h2 < 2; ++h2) {
+                        const int c = 2 * half + h2;  // 32-column chunk of the tile
+                        uint32_t us[32], ud[32], pp[16], pd[16];
+                        tmem_ld32(tmem + lane_off + L::ST_COL + c * 32, us);
+                        tmem_ld32(tmem + lane_off + L::DPT_COL + c * 32, ud);
+                        tmem_wait_ld_dep(us);
+                        tmem_wait_ld_dep(ud);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const int cc = c * 32 + e;
-                        float4 ld;  // (lse, D) of columns cc and cc + 1
-                        asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
-                                     : "=f"(ld.x), "=f"(ld.y), "=f"(ld.z), "=f"(ld.w)
-                                     : "r"(cb + cc * 8));
-                        const bool v0 = cc >= c_lo && cc <= c_hi;
-                        const bool v1 = cc + 1 >= c_lo && cc + 1 <= c_hi;
-                        const float p0 = v0 ? fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - ld.x) : 0.f;
-                        const float p1 = v1 ? fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - ld.z) : 0.f;
-                        pp[e / 2] = pack16(p0, p1, G.core);
-                        pd[e / 2] = pack16(p0 * (__uint_as_float(ud[e]) - ld.y),
-                                           p1 * (__uint_as_float(ud[e + 1]) - ld.w), G.core);
+                        for (int e = 0; e < 32; e += 2) {
+                            const int cc = c * 32 + e;
+                            float4 ld;  // (lse, D) of columns cc and cc + 1
+                            asm volatile("ld.shared.v4.f32 {%0, %1, %2, %3}, [%4];"
+                                         : "=f"(ld.x), "=f"(ld.y), "=f"(ld.z), "=f"(ld.w)
+                                         : "r"(cb + cc * 8));
+                            float p0 = fast_exp2(__uint_as_float(us[e]) * p.scale_log2 - ld.x);
+                            float p1 = fast_exp2(__uint_as_float(us[e + 1]) * p.scale_log2 - ld.z);
+                            if (MASK) {
+                                p0 = cc >= c_lo && cc <= c_hi ? p0 : 0.f;
+                                p1 = cc + 1 >= c_lo && cc + 1 <= c_hi ? p1 : 0.f;
+                            }
+                            const float d0 = p0 * (__uint_as_float(ud[e]) - ld.y);
+                            const float d1 = p1 * (__uint_as_float(ud[e + 1]) - ld.w);
+                            pp[e / 2] = CORE ? pack_f16x2(p0, p1) : pack_bf16x2(p0, p1);
+                            pd[e / 2] = CORE ? pack_f16x2(d0, d1) : pack_bf16x2(d0, d1);
+                        }
+                        // over columns of this half this thread has already read
+                        tmem_st16(tmem + lane_off + L::ST_COL + 64 * half + h2 * 16, pp);
+                        tmem_st16(tmem + lane_off + L::DPT_COL + 64 * half + h2 * 16, pd);
                     }
-                    // over columns this thread has already read
-                    tmem_st16(tmem + lane_off + L::ST_COL + c * 16, pp);
-                    tmem_st16(tmem + lane_off + L::DPT_COL + c * 16, pd);
+                };
+                const bool full =
+                    __all_sync(0xffffffffu, c_lo <= 64 * half && c_hi >= 64 * half + 63);
+                if (G.core) {
+                    if (full)
+                        elementwise(std::true_type{}, std::false_type{});
+                    else
+                        elementwise(std::true_type{}, std::true_type{});
+                } else {
+                    if (full)
+                        elementwise(std::false_type{}, std::false_type{});
+                    else
+                        elementwise(std::false_type{}, std::true_type{});
                 }
                 tmem_wait_st();
                 tc_fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&bars->p_full);
+                if (lane == 0) mbar_arrive(&bars->hp_full[half]);
             }
             if (!ok) break;
             // epilogue: dK = (sum dS^T Q) / sqrt(d), dV = sum P^T dO
-            if (!(ok = bw_warp_wait(&bars->mm_done, (it - 1) & 1, bars))) break;
+            // the last tile's second-half products (and all before them)
+            if (!(ok = bw_warp_wait(&bars->hmm_done[1], (it - 1) & 1, bars))) break;
             tc_fence_after_sync();
             const int64_t krow = (static_cast<int64_t>(G.b) * p.Hkv + G.h) * (G.core ? p.m : p.T) + key;
             float *dKo = (G.core ? p.dKc : p.dK) + krow * D;
             float *dVo = (G.core ? p.dVc : p.dV) + krow * D;
 #pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
+            for (int h2 = 0; h2 < D / 64; ++h2) {
+                const int c = half * (D / 64) + h2;
                 uint32_t uk[32], uv[32];
                 tmem_ld32_wait(tmem + lane_off + L::DK_COL + c * 32, uk);
                 tmem_ld32_wait(tmem + lane_off + L::DV_COL + c * 32, uv);
                 if (!kvalid) continue;
                 if (G.core) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        atomicAdd(dKo + c * 32 + e, __uint_as_float(uk[e]) * p.scale);
-                        atomicAdd(dVo + c * 32 + e, __uint_as_float(uv[e]));
+                    for (int q = 0; q < 8; ++q) {
+                        red_add_v4(dKo + c * 32 + 4 * q, __uint_as_float(uk[4 * q]) * p.scale,
+                                   __uint_as_float(uk[4 * q + 1]) * p.scale,
+                                   __uint_as_float(uk[4 * q + 2]) * p.scale,
+                                   __uint_as_float(uk[4 * q + 3]) * p.scale);
+                        red_add_v4(dVo + c * 32 + 4 * q, __uint_as_float(uv[4 * q]),
+                                   __uint_as_float(uv[4 * q + 1]), __uint_as_float(uv[4 * q + 2]),
+                                   __uint_as_float(uv[4 * q + 3]));
                     }
                 } else {
 #pragma unroll
@@ -830,7 +932,7 @@ __global__ void __launch_bounds__(192, 1)
     }
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 4) {
+    if (warp == kDkvTmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
@@ -1045,7 +1147,8 @@ cudaError_t launch_bw(const void *Q, const void *K, const void *V, const void *K
         if ((e = cudaFuncSetAttribute(bw_dkv_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                       LK::SMEM)) != cudaSuccess)
             return e;
-        bw_dkv_kernel<D><<<grid, 192, LK::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc, mVc, p);
+        bw_dkv_kernel<D><<<grid, kDkvThreads, LK::SMEM, s>>>(mQ, mO, mQ16, mO16, mK, mV, mKc,
+                                                              mVc, p);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     // 4. the pooling
