@@ -141,11 +141,6 @@ __device__ __forceinline__ void red_add_v4(float *ptr, float a, float b, float c
                  : "memory");
 }
 
-__device__ __forceinline__ uint32_t pack16(float a, float b, bool f16)
-{
-    return f16 ? pack_f16x2(a, b) : pack_bf16x2(a, b);
-}
-
 // 1. D = rowsum(dO * O) and the fp16 copies --------------------------------
 
 template <int D, bool OF32>
@@ -735,48 +730,62 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
             const uint64_t dOm = smem_desc_sw128(smem_addr(sO), T::BOX_BYTES, 1024);
             constexpr uint32_t kTile16 = T::TILE_BYTES >> 4;
             constexpr uint32_t kHalf16 = (64 * 128) >> 4;  // 64 rows of a swizzled box
-            uint32_t qc = 0, it = 0, kvc = 0;
+            // Per half h of tile n (tiles numbered over this CTA's items, Q
+            // stage n % QST): A(h, n) issues S^T, dP^T; B(h, n) issues
+            // dV += P^T dO, dK += dS^T Q.  Order within an item:
+            //   A(0,0) A(1,0) | B(0,n) A(0,n+1) B(1,n) A(1,n+1) | ...
+            // so each half runs its own chain and the halves overlap.  A(h,
+            // n+1) waits until B(h, n) has read the half's P^T, dS^T.  No
+            // look-ahead across items: the next item's K, V tiles reuse the
+            // one key-side buffer.
+            uint32_t kvc = 0, base = 0;
             int k = 0;
             bool ok = true;
             for (int item = blockIdx.x; ok && item < n_items; item += gridDim.x, ++k) {
                 const KGeom G = k_geom(item, p);
                 const uint32_t ids = G.core ? id_s_h : id_s_bf, ida = G.core ? id_a_h : id_a_bf;
+                auto issue_a = [&](int h, uint32_t n) -> bool {
+                    if (n > 0 && !bw_lane_wait(&bars->hmm_done[h], (n - 1) & 1, bars)) return false;
+                    tc_fence_after_sync();
+                    const uint32_t s = n % L::QST;
+                    mma_kk<D>(tmem + L::ST_COL + 64 * h, dk, dq + s * kTile16 + h * kHalf16, ids);
+                    mma_kk<D>(tmem + L::DPT_COL + 64 * h, dv, dO + s * kTile16 + h * kHalf16, ids);
+                    mma_commit(&bars->hs_full[h]);
+                    return true;
+                };
+                auto issue_b = [&](int h, uint32_t n, bool first_tile) -> bool {
+                    if (!bw_lane_wait(&bars->hp_full[h], n & 1, bars)) return false;
+                    if (h == 0 && first_tile && k > 0 &&
+                        !bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars))
+                        return false;
+                    tc_fence_after_sync();
+                    const uint32_t s = n % L::QST;
+                    const bool first = first_tile && h == 0;
+                    mma_tm64(tmem + L::DV_COL, tmem + L::ST_COL + 64 * h,
+                             dOm + s * kTile16 + h * 512, ida, first);
+                    mma_tm64(tmem + L::DK_COL, tmem + L::DPT_COL + 64 * h,
+                             dqm + s * kTile16 + h * 512, ida, first);
+                    mma_commit(&bars->hmm_done[h]);
+                    return true;
+                };
+                auto q_ready = [&](uint32_t n) {
+                    return bw_lane_wait(&bars->q_full[n % L::QST], (n / L::QST) & 1, bars);
+                };
                 if (!(ok = bw_lane_wait(&bars->kv_full, kvc & 1, bars))) break;
                 ++kvc;
                 const int n_tiles = p.r * (G.qb - G.qa);
-                for (int i = 0; ok && i < n_tiles; ++i, ++it) {
-                    const uint32_t s = qc % L::QST;
-                    if (!(ok = bw_lane_wait(&bars->q_full[s], (qc / L::QST) & 1, bars))) break;
-                    // S^T, dP^T of both halves; half h waits until the
-                    // previous tile's dV, dK products have read its P^T, dS^T
-                    for (int h = 0; ok && h < 2; ++h) {
-                        if (it > 0 && !(ok = bw_lane_wait(&bars->hmm_done[h], (it - 1) & 1, bars)))
-                            break;
-                        tc_fence_after_sync();
-                        mma_kk<D>(tmem + L::ST_COL + 64 * h, dk, dq + s * kTile16 + h * kHalf16, ids);
-                        mma_kk<D>(tmem + L::DPT_COL + 64 * h, dv, dO + s * kTile16 + h * kHalf16,
-                                  ids);
-                        mma_commit(&bars->hs_full[h]);
-                    }
-                    // dV += P^T dO, dK += dS^T Q, half by half
-                    for (int h = 0; ok && h < 2; ++h) {
-                        if (!(ok = bw_lane_wait(&bars->hp_full[h], it & 1, bars))) break;
-                        if (h == 0 && i == 0 && k > 0 &&
-                            !(ok = bw_lane_wait(&bars->acc_empty, (k - 1) & 1, bars)))
-                            break;
-                        tc_fence_after_sync();
-                        const bool first = i == 0 && h == 0;
-                        mma_tm64(tmem + L::DV_COL, tmem + L::ST_COL + 64 * h,
-                                 dOm + s * kTile16 + h * 512, ida, first);
-                        mma_tm64(tmem + L::DK_COL, tmem + L::DPT_COL + 64 * h,
-                                 dqm + s * kTile16 + h * 512, ida, first);
-                        mma_commit(&bars->hmm_done[h]);
-                    }
-                    if (!ok) break;
-                    mma_commit(&bars->q_empty[s]);
-                    ++qc;
+                if (!(ok = q_ready(base) && issue_a(0, base) && issue_a(1, base))) break;
+                for (int i = 0; ok && i < n_tiles; ++i) {
+                    const uint32_t n = base + i;
+                    const bool more = i + 1 < n_tiles;
+                    if (!(ok = issue_b(0, n, i == 0))) break;
+                    if (more && !(ok = q_ready(n + 1) && issue_a(0, n + 1))) break;
+                    if (!(ok = issue_b(1, n, i == 0))) break;
+                    mma_commit(&bars->q_empty[n % L::QST]);
+                    if (more && !(ok = issue_a(1, n + 1))) break;
                 }
                 if (!ok) break;
+                base += n_tiles;
                 mma_commit(&bars->kv_empty);
             }
             mma_commit(&bars->drain);
