@@ -955,103 +955,183 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
 //   dK_g += a dKc,  dV_g += a dVc,  da = Kg dKc + Vg dVc,
 //   per head k: dz = s_k (da/r - s_k . da/r),
 //   dq_k += (sum_i dz_i Kg_i) / sqrt(d),  dK_g += dz q_k / sqrt(d).
+// Three passes over the group: scores and da (K, V rows read once from
+// DRAM, 8 rows in flight), one read-modify-write of each dK, dV row, then
+// dq per head (key rows again, now from L1).
+template <int D>
+struct BwVec;
+template <>
+struct BwVec<128> {
+    using H = uint2;   // 4 bf16
+    using F = float4;  // 4 fp32
+    static __device__ __forceinline__ void h2f(H v, float (&f)[4])
+    {
+        f[0] = bf16_lo(v.x); f[1] = bf16_hi(v.x); f[2] = bf16_lo(v.y); f[3] = bf16_hi(v.y);
+    }
+    static __device__ __forceinline__ void ld(const float *p, float (&f)[4])
+    {
+        const float4 v = *reinterpret_cast<const float4 *>(p);
+        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&f)[4])
+    {
+        *reinterpret_cast<float4 *>(p) = make_float4(f[0], f[1], f[2], f[3]);
+    }
+};
+template <>
+struct BwVec<64> {
+    using H = uint32_t;  // 2 bf16
+    using F = float2;
+    static __device__ __forceinline__ void h2f(H v, float (&f)[2])
+    {
+        f[0] = bf16_lo(v); f[1] = bf16_hi(v);
+    }
+    static __device__ __forceinline__ void ld(const float *p, float (&f)[2])
+    {
+        const float2 v = *reinterpret_cast<const float2 *>(p);
+        f[0] = v.x; f[1] = v.y;
+    }
+    static __device__ __forceinline__ void st(float *p, const float (&f)[2])
+    {
+        *reinterpret_cast<float2 *>(p) = make_float2(f[0], f[1]);
+    }
+};
+
 template <int D>
 __global__ void bw_pool_kernel(const uint16_t *__restrict__ Q, const uint16_t *__restrict__ K,
                                const uint16_t *__restrict__ V, const BwParams p)
 {
     constexpr int DPL = D / 32;
+    using W = BwVec<D>;
+    using H = typename W::H;
     extern __shared__ float pool_bw_smem[];
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int nwarp = blockDim.x >> 5;
-    float *sc = pool_bw_smem + warp * (p.r + 1) * p.g;  // [r][g] softmax, then [g] da
+    const int r = p.r, g = p.g;
+    float *sc = pool_bw_smem + warp * (r + 2) * g;  // [r][g] softmax, then dz
+    float *da = sc + r * g;                         // [g]
+    float *aw = da + g;                             // [g] pooling weights
+    const float inv_r = 1.0f / static_cast<float>(r);
     const int64_t n_groups = static_cast<int64_t>(p.B) * p.Hkv * p.m;
     for (int64_t gid = static_cast<int64_t>(blockIdx.x) * nwarp + warp; gid < n_groups;
          gid += static_cast<int64_t>(gridDim.x) * nwarp) {
         const int64_t pair = gid / p.m, j = gid - pair * p.m;
         const int64_t b = pair / p.Hkv, h = pair - b * p.Hkv;
-        const int64_t row0 = pair * p.T + j * p.g;  // first key row of the group
-        const int64_t last = j * p.g + p.g - 1;
+        const int64_t row0 = pair * p.T + j * g;  // first key row of the group
+        const int64_t last = j * g + g - 1;
+        const int64_t lo = lane * DPL;
+        auto qrow = [&](int k) { return ((b * p.Hq + h * r + k) * p.T + last) * D; };
         float dkc[DPL], dvc[DPL];
+        W::ld(p.dKc + (pair * p.m + j) * D + lo, dkc);
+        W::ld(p.dVc + (pair * p.m + j) * D + lo, dvc);
+        // pass 1: logits of every head, da_i = (K_i . dKc + V_i . dVc) / r
+        for (int i0 = 0; i0 < g; i0 += 8) {
+            H kv[8], vv[8];
 #pragma unroll
-        for (int e = 0; e < DPL; ++e) {
-            dkc[e] = p.dKc[(pair * p.m + j) * D + lane * DPL + e];
-            dvc[e] = p.dVc[(pair * p.m + j) * D + lane * DPL + e];
-        }
-        // scores and softmax per query head
-        for (int k = 0; k < p.r; ++k) {
-            const uint16_t *q = Q + ((b * p.Hq + h * p.r + k) * p.T + last) * D + lane * DPL;
-            float qf[DPL];
-#pragma unroll
-            for (int e = 0; e < DPL; ++e) qf[e] = __uint_as_float(static_cast<uint32_t>(q[e]) << 16);
-            float mx = -INFINITY;
-            for (int i = 0; i < p.g; ++i) {
-                const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
-                float s = 0.f;
-#pragma unroll
-                for (int e = 0; e < DPL; ++e)
-                    s = fmaf(qf[e], __uint_as_float(static_cast<uint32_t>(kr[e]) << 16), s);
-                s = warp_sum(s) * p.scale_log2;
-                if (lane == 0) sc[k * p.g + i] = s;
-                mx = fmaxf(mx, s);
+            for (int u = 0; u < 8; ++u) {
+                if (i0 + u < g) {
+                    kv[u] = *reinterpret_cast<const H *>(K + (row0 + i0 + u) * D + lo);
+                    vv[u] = *reinterpret_cast<const H *>(V + (row0 + i0 + u) * D + lo);
+                }
             }
-            __syncwarp();
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                if (i0 + u < g) {
+                    float kf[DPL], vf[DPL];
+                    W::h2f(kv[u], kf);
+                    W::h2f(vv[u], vf);
+                    float t = 0.f;
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) t = fmaf(kf[e], dkc[e], fmaf(vf[e], dvc[e], t));
+                    t = warp_sum(t);
+                    if (lane == 0) da[i0 + u] = t * inv_r;
+                }
+            }
+            for (int k = 0; k < r; ++k) {
+                float qf[DPL];
+                W::h2f(*reinterpret_cast<const H *>(Q + qrow(k) + lo), qf);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    if (i0 + u < g) {
+                        float kf[DPL];
+                        W::h2f(kv[u], kf);
+                        float t = 0.f;
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) t = fmaf(qf[e], kf[e], t);
+                        t = warp_sum(t);
+                        if (lane == 0) sc[k * g + i0 + u] = t * p.scale_log2;
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        // softmax per head, weights a = mean over heads, then dz in place
+        for (int i = lane; i < g; i += 32) aw[i] = 0.f;
+        __syncwarp();
+        for (int k = 0; k < r; ++k) {
+            float mx = -INFINITY;
+            for (int i = lane; i < g; i += 32) mx = fmaxf(mx, sc[k * g + i]);
+            mx = warp_max(mx);
             float sum = 0.f;
-            for (int i = lane; i < p.g; i += 32) {
-                const float e = exp2f(sc[k * p.g + i] - mx);
-                sc[k * p.g + i] = e;
+            for (int i = lane; i < g; i += 32) {
+                const float e = exp2f(sc[k * g + i] - mx);
+                sc[k * g + i] = e;
                 sum += e;
             }
             sum = warp_sum(sum);
-            __syncwarp();
-            for (int i = lane; i < p.g; i += 32) sc[k * p.g + i] /= sum;
+            const float inv = 1.0f / sum;
+            float sd = 0.f;
+            for (int i = lane; i < g; i += 32) {
+                const float sv = sc[k * g + i] * inv;
+                sc[k * g + i] = sv;
+                aw[i] += sv * inv_r;
+                sd += sv * da[i];
+            }
+            sd = warp_sum(sd);
+            for (int i = lane; i < g; i += 32) sc[k * g + i] *= da[i] - sd;  // dz
             __syncwarp();
         }
-        // dK_g, dV_g through the weights; da_i
-        float *da = sc + p.r * p.g;
-        const float inv_r = 1.0f / static_cast<float>(p.r);
-        for (int i = 0; i < p.g; ++i) {
-            float a = 0.f;
-            for (int k = 0; k < p.r; ++k) a += sc[k * p.g + i];
-            a *= inv_r;
-            const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
-            const uint16_t *vr = V + (row0 + i) * D + lane * DPL;
-            float *dkr = p.dK + (row0 + i) * D + lane * DPL;
-            float *dvr = p.dV + (row0 + i) * D + lane * DPL;
-            float s = 0.f;
+        // pass 2: dK_i += a_i dKc + (sum_k dz_ki q_k) / sqrt(d), dV_i += a_i dVc
+        for (int i = 0; i < g; ++i) {
+            float dk[DPL], dv[DPL];
+            float *dkr = p.dK + (row0 + i) * D + lo;
+            float *dvr = p.dV + (row0 + i) * D + lo;
+            W::ld(dkr, dk);
+            W::ld(dvr, dv);
+            const float a = aw[i];
 #pragma unroll
             for (int e = 0; e < DPL; ++e) {
-                s = fmaf(__uint_as_float(static_cast<uint32_t>(kr[e]) << 16), dkc[e], s);
-                s = fmaf(__uint_as_float(static_cast<uint32_t>(vr[e]) << 16), dvc[e], s);
-                dkr[e] += a * dkc[e];
-                dvr[e] += a * dvc[e];
+                dk[e] = fmaf(a, dkc[e], dk[e]);
+                dv[e] = fmaf(a, dvc[e], dv[e]);
             }
-            s = warp_sum(s);
-            if (lane == 0) da[i] = s * inv_r;
+            for (int k = 0; k < r; ++k) {
+                float qf[DPL];
+                W::h2f(*reinterpret_cast<const H *>(Q + qrow(k) + lo), qf);
+                const float c = sc[k * g + i] * p.scale;
+#pragma unroll
+                for (int e = 0; e < DPL; ++e) dk[e] = fmaf(c, qf[e], dk[e]);
+            }
+            W::st(dkr, dk);
+            W::st(dvr, dv);
         }
-        __syncwarp();
-        // through each head's softmax to its query and the keys
-        for (int k = 0; k < p.r; ++k) {
-            float sd = 0.f;
-            for (int i = lane; i < p.g; i += 32) sd += sc[k * p.g + i] * da[i];
-            sd = warp_sum(sd);
-            const int64_t qrow = (b * p.Hq + h * p.r + k) * p.T + last;
-            const uint16_t *q = Q + qrow * D + lane * DPL;
+        // pass 3: dq_k += (sum_i dz_ki K_i) / sqrt(d)
+        for (int k = 0; k < r; ++k) {
             float dq[DPL];
 #pragma unroll
             for (int e = 0; e < DPL; ++e) dq[e] = 0.f;
-            for (int i = 0; i < p.g; ++i) {
-                const float dz = sc[k * p.g + i] * (da[i] - sd);
-                const uint16_t *kr = K + (row0 + i) * D + lane * DPL;
-                float *dkr = p.dK + (row0 + i) * D + lane * DPL;
+            for (int i = 0; i < g; ++i) {
+                float kf[DPL];
+                W::h2f(*reinterpret_cast<const H *>(K + (row0 + i) * D + lo), kf);
+                const float c = sc[k * g + i];
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) {
-                    dq[e] = fmaf(dz, __uint_as_float(static_cast<uint32_t>(kr[e]) << 16), dq[e]);
-                    dkr[e] += dz * p.scale * __uint_as_float(static_cast<uint32_t>(q[e]) << 16);
-                }
+                for (int e = 0; e < DPL; ++e) dq[e] = fmaf(c, kf[e], dq[e]);
             }
-            float *dqr = p.dQ + qrow * D + lane * DPL;
+            float *dqr = p.dQ + qrow(k) + lo;
+            float cur[DPL];
+            W::ld(dqr, cur);
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) dqr[e] += dq[e] * p.scale;
+            for (int e = 0; e < DPL; ++e) cur[e] = fmaf(dq[e], p.scale, cur[e]);
+            W::st(dqr, cur);
         }
         __syncwarp();
     }
@@ -1162,8 +1242,11 @@ cudaError_t launch_bw(const void *Q, const void *K, const void *V, const void *K
     }
     // 4. the pooling
     if (m > 0) {
-        const int warps = 8;
-        const size_t smem = sizeof(float) * warps * (p.r + 1) * g;
+        // 8 warps per block, fewer when a warp's scratch is large (r, g)
+        const size_t per_warp = sizeof(float) * (p.r + 2) * g;
+        int warps = 8;
+        while (warps > 1 && per_warp * warps > 200 * 1024) --warps;
+        const size_t smem = per_warp * warps;
         const int64_t groups = static_cast<int64_t>(B) * Hkv * m;
         const int64_t want = (groups + warps - 1) / warps;
         const int blocks = static_cast<int>(want < 148LL * 16 ? want : 148LL * 16);

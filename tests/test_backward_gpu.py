@@ -28,6 +28,8 @@ CASES = [
     (1, 2, 2, 100, 64, 16, 1000),    # window wider than the sequence: no core
     (1, 4, 1, 333, 64, 8, 40),       # r = 4, T mod g != 0
     (2, 2, 1, 2500, 64, 8, 64),      # three core tiles, chunked query ranges
+    (1, 8, 1, 700, 128, 32, 64),     # r = 8, g = 32
+    (1, 24, 1, 600, 64, 256, 64),    # r = 24, g = 256: pooling scratch for 7 warps a block
 ]
 
 
