@@ -896,7 +896,14 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
             }
             if (!ok) break;
             // epilogue: dK = (sum dS^T Q) / sqrt(d), dV = sum P^T dO
-            // the last tile's second-half products (and all before them)
+            // The last tile's products.  A parity wait is sound only when
+            // the phase before the awaited one is known to be complete.
+            // Half 0's first: each group has seen the last tile's S^T of its
+            // own half issued, A(1, last) follows A(0, last), and A(0, last)
+            // is issued only once half 0's phase last - 1 is complete.
+            // Then half 1's: B(0, last) follows B(1, last - 1), so its
+            // completion implies half 1's phase last - 1.
+            if (!(ok = bw_warp_wait(&bars->hmm_done[0], (it - 1) & 1, bars))) break;
             if (!(ok = bw_warp_wait(&bars->hmm_done[1], (it - 1) & 1, bars))) break;
             tc_fence_after_sync();
             const int64_t krow = (static_cast<int64_t>(G.b) * p.Hkv + G.h) * (G.core ? p.m : p.T) + key;
