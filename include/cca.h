@@ -115,7 +115,7 @@ cca_status cca_pool(const void *Q, const void *K, const void *V, void *Kc,
  * and 全局-局部模块可微融合).
  *   Q [B, Hq, T, d], K, V [B, Hkv, T, d] (bf16), Kc, Vc [B, Hkv, m, d]
  *   (fp16, from cca_pool), O [B, Hq, T, d] written in o_dtype (bf16 or
- *   fp32).
+ *   fp32), 32-byte aligned (CCA_ERR_INVALID_ARG otherwise).
  * O[t] = softmax over { q_t . Kc[j] / sqrt(d) : j < ws(t)/g } and
  * { q_t . K[i] / sqrt(d) : ws(t) <= i <= t } applied to [Vc ; V].
  * Runs on tcgen05 tensor cores with TMA-staged tiles.
@@ -153,7 +153,8 @@ size_t cca_attn_backward_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int 
  * query and its keys).
  *   Q, K, V, Kc, Vc as for cca_attn_prefill; O and lse from
  *   cca_attn_prefill_lse on the same inputs (O in o_dtype); dO [B, Hq, T, d]
- *   bf16.  dQ [B, Hq, T, d], dK, dV [B, Hkv, T, d]: fp32, written.
+ *   bf16.  dQ [B, Hq, T, d], dK, dV [B, Hkv, T, d]: fp32, written, each
+ *   32-byte aligned (CCA_ERR_INVALID_ARG otherwise).
  *   workspace: cca_attn_backward_workspace_bytes bytes of device memory,
  *   256-byte aligned (fp16 copies of Q and dO, per-row sums, fp32 core
  *   gradients; the call clears what it accumulates).  r = Hq / Hkv <= 32.

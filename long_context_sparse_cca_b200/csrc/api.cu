@@ -101,6 +101,8 @@ cca_status cca_attn_prefill(const void *Q, const void *K, const void *V, const v
     if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(O, any) ||
         !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
         return CCA_ERR_INVALID_ARG;
+    if (any && (reinterpret_cast<uintptr_t>(O) & 31u) != 0)
+        return CCA_ERR_INVALID_ARG;  // output rows are written with 32-byte stores
     if (!any) return CCA_OK;
     const int64_t n_items = ((T + 255) / 256) * int64_t(B) * Hq;
     if (n_items > INT32_MAX) return CCA_ERR_UNSUPPORTED;
@@ -128,6 +130,8 @@ cca_status cca_attn_prefill_lse(const void *Q, const void *K, const void *V, con
     if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(O, any) ||
         !ptr_ok(lse, any) || !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
         return CCA_ERR_INVALID_ARG;
+    if (any && (reinterpret_cast<uintptr_t>(O) & 31u) != 0)
+        return CCA_ERR_INVALID_ARG;  // output rows are written with 32-byte stores
     if (!any) return CCA_OK;
     const int64_t n_items = ((T + 255) / 256) * int64_t(B) * Hq;
     if (n_items > INT32_MAX) return CCA_ERR_UNSUPPORTED;
@@ -167,6 +171,10 @@ cca_status cca_attn_backward(const void *Q, const void *K, const void *V, const 
     if (!ptr_ok(Q, any) || !ptr_ok(K, any) || !ptr_ok(V, any) || !ptr_ok(O, any) ||
         !ptr_ok(lse, any) || !ptr_ok(dO, any) || !ptr_ok(dQ, any) || !ptr_ok(dK, any) ||
         !ptr_ok(dV, any) || !ptr_ok(Kc, m > 0) || !ptr_ok(Vc, m > 0))
+        return CCA_ERR_INVALID_ARG;
+    // the gradient rows are written with 32-byte stores
+    if (any && ((reinterpret_cast<uintptr_t>(dQ) | reinterpret_cast<uintptr_t>(dK) |
+                 reinterpret_cast<uintptr_t>(dV)) & 31u) != 0)
         return CCA_ERR_INVALID_ARG;
     if (!any) return CCA_OK;
     if (workspace == nullptr || (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0 ||

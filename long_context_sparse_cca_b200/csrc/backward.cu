@@ -132,6 +132,18 @@ __device__ __forceinline__ void mma_tm(uint32_t d_tmem, uint32_t a_tmem, uint64_
         mma_ts(d_tmem, a_tmem + kk * 8, b0 + kk * 128, idesc, (first && kk == 0) ? 0u : 1u);
 }
 
+// Eight fp32 values x[0..8) * scale to global memory in one 32-byte store
+// (p 32-byte aligned): a thread writing its own row fills whole sectors.
+__device__ __forceinline__ void st_global_x8(float *ptr, const uint32_t *x, float scale)
+{
+    asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(ptr),
+                 "f"(__uint_as_float(x[0]) * scale), "f"(__uint_as_float(x[1]) * scale),
+                 "f"(__uint_as_float(x[2]) * scale), "f"(__uint_as_float(x[3]) * scale),
+                 "f"(__uint_as_float(x[4]) * scale), "f"(__uint_as_float(x[5]) * scale),
+                 "f"(__uint_as_float(x[6]) * scale), "f"(__uint_as_float(x[7]) * scale)
+                 : "memory");
+}
+
 // Four fp32 additions to global memory in one 16-byte reduction (p 16-byte
 // aligned); the order among concurrent adders is unspecified.
 __device__ __forceinline__ void red_add_v4(float *ptr, float a, float b, float c, float d)
@@ -523,13 +535,9 @@ __global__ void __launch_bounds__(kDqThreads, 1)
                 uint32_t u[32];
                 tmem_ld32_wait(tmem + lane_off + L::DQ_COL + c * 32, u);
                 if (valid) {
-                    float4 *dst = reinterpret_cast<float4 *>(p.dQ + qrow * D + c * 32);
 #pragma unroll
-                    for (int q = 0; q < 8; ++q)
-                        dst[q] = make_float4(__uint_as_float(u[4 * q]) * p.scale,
-                                             __uint_as_float(u[4 * q + 1]) * p.scale,
-                                             __uint_as_float(u[4 * q + 2]) * p.scale,
-                                             __uint_as_float(u[4 * q + 3]) * p.scale);
+                    for (int q = 0; q < 4; ++q)
+                        st_global_x8(p.dQ + qrow * D + c * 32 + 8 * q, u + 8 * q, p.scale);
                 }
             }
             tc_fence_before_sync();
@@ -929,15 +937,9 @@ __global__ void __launch_bounds__(kDkvThreads, 1)
                     }
                 } else {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        reinterpret_cast<float4 *>(dKo + c * 32)[q] =
-                            make_float4(__uint_as_float(uk[4 * q]) * p.scale,
-                                        __uint_as_float(uk[4 * q + 1]) * p.scale,
-                                        __uint_as_float(uk[4 * q + 2]) * p.scale,
-                                        __uint_as_float(uk[4 * q + 3]) * p.scale);
-                        reinterpret_cast<float4 *>(dVo + c * 32)[q] =
-                            make_float4(__uint_as_float(uv[4 * q]), __uint_as_float(uv[4 * q + 1]),
-                                        __uint_as_float(uv[4 * q + 2]), __uint_as_float(uv[4 * q + 3]));
+                    for (int q = 0; q < 4; ++q) {
+                        st_global_x8(dKo + c * 32 + 8 * q, uk + 8 * q, p.scale);
+                        st_global_x8(dVo + c * 32 + 8 * q, uv + 8 * q, 1.0f);
                     }
                 }
             }

@@ -79,6 +79,7 @@ def test_prefill_argument_checks(L):
     assert call(T=0, O=0) == cca.CCA_OK  # empty sequence
     assert call(Kc=0) == cca.CCA_ERR_INVALID_ARG  # T // g > 0 needs Kc
     assert call(Kc=FAKE + (1 << 20) + 8) == cca.CCA_ERR_INVALID_ARG  # misaligned
+    assert call(O=FAKE + (1 << 24) + 16) == cca.CCA_ERR_INVALID_ARG  # O not 32-byte aligned
 
 
 def _cache(B=1, Hq=2, Hkv=2, d=128, g=16, w=64, core_cap=8, tail_cap=80, length=0,
@@ -280,3 +281,32 @@ def test_lca_argument_checks(L):
     assert L.cca_lca_cache_prefill(ctypes.byref(c), P(QS), P(FAKE), P(FAKE), P(FAKE), 20, 130,
                                    None) == cca.CCA_ERR_INVALID_ARG
     assert c.len == 0
+
+
+def test_backward_argument_checks(L):
+    """cca_attn_backward refuses bad shapes, outputs that are not 32-byte
+    aligned, a short workspace and aliasing, all before any launch."""
+    P = ctypes.c_void_p
+    B, Hq, Hkv, T, d, g, w = 1, 2, 2, 256, 128, 16, 64
+    nb = L.cca_attn_backward_workspace_bytes(B, Hq, Hkv, T, d, g)
+    assert nb > 0
+    base = FAKE
+    step = 1 << 24  # every buffer 16 MiB apart: no overlaps unless asked
+    names = ("Q", "K", "V", "Kc", "Vc", "O", "lse", "dO", "dQ", "dK", "dV", "ws")
+    addr = {n: base + i * step for i, n in enumerate(names)}
+
+    def call(**kw):
+        a = dict(addr)
+        a.update({k: v for k, v in kw.items() if k in addr})
+        return L.cca_attn_backward(P(a["Q"]), P(a["K"]), P(a["V"]), P(a["Kc"]), P(a["Vc"]),
+                                   P(a["O"]), 0, P(a["lse"]), P(a["dO"]), P(a["dQ"]), P(a["dK"]),
+                                   P(a["dV"]), B, kw.get("Hq", Hq), Hkv, T, d, g, w,
+                                   P(a["ws"]), kw.get("nb", nb), None)
+
+    assert call(dK=addr["dK"] + 16) == cca.CCA_ERR_INVALID_ARG   # 16- but not 32-byte aligned
+    assert call(dQ=addr["dQ"] + 16) == cca.CCA_ERR_INVALID_ARG
+    assert call(ws=addr["ws"] + 128) == cca.CCA_ERR_INVALID_ARG  # workspace 256-byte aligned
+    assert call(nb=nb - 1) == cca.CCA_ERR_INVALID_ARG
+    assert call(dV=addr["Q"]) == cca.CCA_ERR_INVALID_ARG          # output aliases an input
+    assert call(Hq=3) == cca.CCA_ERR_INVALID_ARG                  # Hq % Hkv != 0
+    assert call(Hq=66) == cca.CCA_ERR_UNSUPPORTED                 # r = 33 > 32
