@@ -310,3 +310,35 @@ def test_backward_argument_checks(L):
     assert call(dV=addr["Q"]) == cca.CCA_ERR_INVALID_ARG          # output aliases an input
     assert call(Hq=3) == cca.CCA_ERR_INVALID_ARG                  # Hq % Hkv != 0
     assert call(Hq=66) == cca.CCA_ERR_UNSUPPORTED                 # r = 33 > 32
+
+
+class _FakeCuda:
+    """A stand-in for a contiguous CUDA tensor: enough for the binding's
+    argument checks, which run before any library call."""
+
+    def __init__(self, shape, dtype):
+        self.shape, self.dtype, self.is_cuda = shape, dtype, True
+
+    def is_contiguous(self):
+        return True
+
+    def data_ptr(self):
+        return FAKE
+
+
+def test_core_rows_are_fp16():
+    """Core keys/values (Kc, Vc and the cache's core slots) are fp16: the
+    header names that layout and the binding refuses bf16 core rows before
+    calling the library."""
+    import torch
+    with open(os.path.join(ROOT, "include", "cca.h")) as f:
+        text = f.read()
+    assert "Kc, Vc [B, Hkv, m, d], m = floor(T / g)  (fp16, written)" in text
+    assert "(fp16, from cca_pool)" in text
+    B, H, T, d, g = 1, 2, 64, 128, 16
+    qkv = [_FakeCuda((B, H, T, d), torch.bfloat16) for _ in range(3)]
+    bad = _FakeCuda((B, H, T // g, d), torch.bfloat16)
+    with pytest.raises(ValueError, match="float16"):
+        cca.cca_pool(*qkv, g, Kc=bad, Vc=bad)
+    with pytest.raises(ValueError, match="float16"):
+        cca.cca_attn_prefill(*qkv, bad, bad, g, 64, O=_FakeCuda((B, H, T, d), torch.bfloat16))
