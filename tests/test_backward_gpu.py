@@ -93,3 +93,36 @@ def test_backward_repeatable(cca):
     assert cca.cca_device_status() == cca.CCA_OK
     for x, y in zip(a, b):
         assert float((x - y).abs().max()) <= 1e-5 * float(x.abs().max())
+
+
+def test_backward_poisoned_buffers(cca):
+    """Outputs pre-filled with NaN and a workspace of 0xFF bytes, three calls
+    in a row on a shape with partial key tiles and several core tiles: every
+    gradient element is written, and each call matches the oracle (a read of
+    an accumulator before its last products landed showed up exactly here,
+    on partial key tiles)."""
+    import torch
+    case = (2, 2, 1, 2500, 64, 8, 64)
+    B, Hq, Hkv, T, d, g, w = case
+    seed = 40 + sum(case)
+    q = synth.random_bf16((B, Hq, T, d), seed)
+    k = synth.random_bf16((B, Hkv, T, d), seed + 1, scale=1.5)
+    v = synth.random_bf16((B, Hkv, T, d), seed + 2)
+    do = synth.random_bf16((B, Hq, T, d), seed + 3)
+    Q, K, V, dO = (to_cuda(x) for x in (q, k, v, do))
+    Kc, Vc = cca.cca_pool(Q, K, V, g)
+    O, lse = cca.cca_attn_prefill_lse(Q, K, V, Kc, Vc, g, w)
+    ref = bw.backward(*(synth.bf16_bits_to_f64(x) for x in (q, k, v)), g, w,
+                      synth.bf16_bits_to_f64(do))
+    nb = cca.cca_attn_backward_workspace_bytes(B, Hq, Hkv, T, d, g)
+    for _ in range(3):
+        outs = [torch.full(shape, float("nan"), device="cuda")
+                for shape in ((B, Hq, T, d), (B, Hkv, T, d), (B, Hkv, T, d))]
+        ws = torch.full((nb,), 255, dtype=torch.uint8, device="cuda")
+        cca.cca_attn_backward(Q, K, V, Kc, Vc, O, lse, dO, g, w, *outs, workspace=ws)
+        assert cca.cca_device_status() == cca.CCA_OK
+        for name, a, b in zip(("dQ", "dK", "dV"), outs, ref):
+            a = a.double().cpu().numpy()
+            assert not np.isnan(a).any(), f"{name}: unwritten elements"
+            e = grad_errors(a, b)
+            assert e["ok"], f"{name}: {e}"
