@@ -52,3 +52,43 @@ def test_kv_cache_reduction_at_128k():
     assert c["full_cache_bytes"] == 2 * 32 * 131072 * 128 * 2
     assert c["cca_cache_bytes"] == 2 * 32 * (8192 + 1040) * 128 * 2
     assert abs(c["reduction"] - 0.9296) < 1e-4
+
+
+def test_backward_flops_and_lca_bytes():
+    # backward: 10 d per attended pair (S, dP, dV, dK, dQ at 2 d each)
+    wl = synth.PREFILL_32K
+    assert bench.backward_flops(wl) == pytest.approx(10.0 / 4.0 * bench.prefill_flops(wl))
+    assert bench.backward_flops(wl) == pytest.approx(2.653e12, rel=1e-3)
+    # LCA condensation: every query row, K and V read; Kc, Vc written (2 bytes)
+    w = synth.PREFILL_128K
+    m = w.T // w.g
+    expect = 2 * (w.B * w.Hq * w.T * w.d + 2 * w.B * w.Hkv * w.T * w.d + 2 * w.B * w.Hkv * m * w.d)
+    assert bench.lca_pool_bytes(w) == expect
+    assert bench.lca_pool_bytes(w) == pytest.approx(3.355e9, rel=1e-3)
+    # it reads all queries where CCA's pooling reads one per group
+    assert bench.lca_pool_bytes(w) - bench.pool_bytes(w) == 2 * w.B * w.Hq * (w.T - m) * w.d
+
+
+def test_measured_traffic_is_tied_to_the_kernel_sources(tmp_path, monkeypatch):
+    """A traffic line counts only while the prefill sources hash to the value
+    recorded with it; another workload or a stale hash reads as unmeasured."""
+    h = bench.prefill_source_hash()
+    assert len(h) == 16
+    assert "long_context_sparse_cca_b200/csrc/tma_map.h" in bench.PREFILL_SOURCES
+    prof = tmp_path / "traffic.md"
+    prof.write_text(f"# summary\n`traffic wlA 4.5e9 {h}`\n`traffic wlB 1.0e9 0123456789abcdef`\n")
+    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(prof))
+    assert bench.measured_traffic("wlA") == 4.5e9
+    assert bench.measured_traffic("wlB") is None   # recorded on other sources
+    assert bench.measured_traffic("wlC") is None   # never captured
+    monkeypatch.setattr(bench, "TRAFFIC_PROFILE", str(tmp_path / "missing.md"))
+    assert bench.measured_traffic("wlA") is None
+
+
+def test_committed_traffic_lines_match_the_current_sources():
+    """The committed summary carries a line for each timed prefill workload,
+    taken on the present kernel sources."""
+    for name in (synth.PREFILL_128K.name,) + bench.EXTRA_PREFILL:
+        t = bench.measured_traffic(name)
+        assert t is not None, name
+        assert t >= bench.prefill_bytes(synth.WORKLOADS[name]) * 0.9, name
