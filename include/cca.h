@@ -159,8 +159,9 @@ size_t cca_attn_backward_workspace_bytes(int B, int Hq, int Hkv, int64_t T, int 
  *   256-byte aligned (fp16 copies of Q and dO, per-row sums, fp32 core
  *   gradients; the call clears what it accumulates).  r = Hq / Hkv <= 32.
  * Runs as four launches on `stream` (per-row sums; dQ on tcgen05 tensor
- * cores, one query tile per CTA; dK, dV on tcgen05, one key tile per CTA;
- * the pooling's chain rule, one warp per group).  Errors as
+ * cores, persistent CTAs taking one 128-row query tile at a time; dK, dV on
+ * tcgen05, persistent CTAs taking one 128-key tile at a time; the pooling's
+ * chain rule, one warp per group).  Errors as
  * cca_attn_prefill; values beyond the fp16 range in Q or dO are clamped in
  * the core stream's copies and reported as CCA_ERR_RANGE.
  */
