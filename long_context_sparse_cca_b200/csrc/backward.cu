@@ -1100,28 +1100,48 @@ __global__ void bw_pool_kernel(const uint16_t *__restrict__ Q, const uint16_t *_
             for (int i = lane; i < g; i += 32) sc[k * g + i] *= da[i] - sd;  // dz
             __syncwarp();
         }
-        // pass 2: dK_i += a_i dKc + (sum_k dz_ki q_k) / sqrt(d), dV_i += a_i dVc
-        for (int i = 0; i < g; ++i) {
-            float dk[DPL], dv[DPL];
-            float *dkr = p.dK + (row0 + i) * D + lo;
-            float *dvr = p.dV + (row0 + i) * D + lo;
-            W::ld(dkr, dk);
-            W::ld(dvr, dv);
-            const float a = aw[i];
+        // pass 2: dK_i += a_i dKc + (sum_k dz_ki q_k) / sqrt(d), dV_i += a_i dVc;
+        // four rows' loads in flight before any of them is updated
+        constexpr int RB = 4;
+        for (int i0 = 0; i0 < g; i0 += RB) {
+            float dk[RB][DPL], dv[RB][DPL];
 #pragma unroll
-            for (int e = 0; e < DPL; ++e) {
-                dk[e] = fmaf(a, dkc[e], dk[e]);
-                dv[e] = fmaf(a, dvc[e], dv[e]);
+            for (int u = 0; u < RB; ++u) {
+                if (i0 + u < g) {
+                    W::ld(p.dK + (row0 + i0 + u) * D + lo, dk[u]);
+                    W::ld(p.dV + (row0 + i0 + u) * D + lo, dv[u]);
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < RB; ++u) {
+                if (i0 + u < g) {
+                    const float a = aw[i0 + u];
+#pragma unroll
+                    for (int e = 0; e < DPL; ++e) {
+                        dk[u][e] = fmaf(a, dkc[e], dk[u][e]);
+                        dv[u][e] = fmaf(a, dvc[e], dv[u][e]);
+                    }
+                }
             }
             for (int k = 0; k < r; ++k) {
                 float qf[DPL];
                 W::h2f(*reinterpret_cast<const H *>(Q + qrow(k) + lo), qf);
-                const float c = sc[k * g + i] * p.scale;
 #pragma unroll
-                for (int e = 0; e < DPL; ++e) dk[e] = fmaf(c, qf[e], dk[e]);
+                for (int u = 0; u < RB; ++u) {
+                    if (i0 + u < g) {
+                        const float c = sc[k * g + i0 + u] * p.scale;
+#pragma unroll
+                        for (int e = 0; e < DPL; ++e) dk[u][e] = fmaf(c, qf[e], dk[u][e]);
+                    }
+                }
             }
-            W::st(dkr, dk);
-            W::st(dvr, dv);
+#pragma unroll
+            for (int u = 0; u < RB; ++u) {
+                if (i0 + u < g) {
+                    W::st(p.dK + (row0 + i0 + u) * D + lo, dk[u]);
+                    W::st(p.dV + (row0 + i0 + u) * D + lo, dv[u]);
+                }
+            }
         }
         // pass 3: dq_k += (sum_i dz_ki K_i) / sqrt(d)
         for (int k = 0; k < r; ++k) {
