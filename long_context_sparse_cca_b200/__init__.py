@@ -15,7 +15,10 @@ Entry points (same names as the C ABI):
     cca_attn_decode, cca_decode_step (append + decode in one launch),
     cca_decode_workspace_bytes, cca_attn_decode_noalloc,
     cca_cache_append_rows, cca_attn_decode_rows (per-row lengths in device
-    memory), cca_selftest_wait_timeout, cca_device_status
+    memory), cca_lca_pool, cca_lca_cache_prefill, cca_lca_cache_append (the
+    LCA variant's condensation; ``lca_query_sums`` allocates the running
+    query sums its cache calls keep), cca_selftest_wait_timeout,
+    cca_device_status
 and the ``Cache`` class holding a decode cache's device buffers.
 """
 
