@@ -74,6 +74,8 @@ def _bind(path: str):
     L.cca_oracle_attend_rows.restype = i
     L.cca_oracle_cache_append.argtypes = [ctypes.POINTER(_Cache), P, P, P]
     L.cca_oracle_cache_append.restype = i
+    L.cca_oracle_lca_cache_append.argtypes = [ctypes.POINTER(_Cache), P, P, P, P, i]
+    L.cca_oracle_lca_cache_append.restype = i
     L.cca_oracle_decode.argtypes = [ctypes.POINTER(_Cache), P, P]
     L.cca_oracle_decode.restype = i
     return L
@@ -218,6 +220,16 @@ class Cache:
 
     def append(self, q, k, v) -> None:
         _check(self.try_append(q, k, v), "append")
+
+    def lca_append(self, q_sum: np.ndarray, q, k, v, d_rope: int) -> None:
+        """LCA variant: append one token, condensing the group it completes
+        with the open group's average queries.  q_sum [B,Hq,d] float64, the
+        open group's query sums, is updated in place."""
+        assert q_sum.dtype == np.float64 and q_sum.flags.c_contiguous
+        q, k, v = _f64(q), _f64(k), _f64(v)
+        _check(self._lib.cca_oracle_lca_cache_append(ctypes.byref(self._c), _ptr(q_sum),
+                                                     _ptr(q), _ptr(k), _ptr(v), int(d_rope)),
+               "lca_append")
 
     def decode(self, q) -> np.ndarray:
         q = _f64(q)

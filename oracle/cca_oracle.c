@@ -399,6 +399,88 @@ int cca_oracle_cache_append(cca_oracle_cache *c, const double *q,
     return CCA_ORACLE_OK;
 }
 
+/*
+ * Decode cache of the LCA variant (page "Latent-Condensed Transformer for
+ * Efficient Long Context Modeling", section 2 方法论, 推理流程: the cache
+ * keeps the condensed vectors, their anchors and the newest w tokens, and
+ * condenses old groups as new tokens arrive).
+ *
+ * Reading taken: a group is condensed when its last token arrives, with the
+ * weights and anchor of cca_oracle_lca_pool; its average query needs every
+ * query row of the group, which the cache does not keep, so q_sum
+ * [B, Hq, d] holds the sum of the query rows of the open group per head.
+ * Token t = len: k, v go to ring slot t % tail_cap; if t completes group
+ * j = t / g the group is condensed from the ring with average queries
+ * (q_sum + q) / g into core slot j and q_sum restarts at zero, otherwise q
+ * is added to q_sum.  Then len = t + 1.
+ */
+int cca_oracle_lca_cache_append(cca_oracle_cache *c, double *q_sum, const double *q,
+                                const double *k, const double *v, int d_rope)
+{
+    if (!cache_ok(c) || !q_sum || d_rope < 0 || d_rope > c->d) return CCA_ORACLE_EINVAL;
+    const long t = c->len;
+    const int B = c->B, Hq = c->Hq, Hkv = c->Hkv, d = c->d, g = c->g;
+    const int r = Hq / Hkv;
+    if (t / g >= c->core_cap) return CCA_ORACLE_ECAPACITY;
+    const long slot = t % c->tail_cap;
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            const size_t kv = (size_t)b * Hkv + h;
+            memcpy(c->k_tail + (kv * c->tail_cap + slot) * d, k + kv * d, sizeof(double) * d);
+            memcpy(c->v_tail + (kv * c->tail_cap + slot) * d, v + kv * d, sizeof(double) * d);
+        }
+    const size_t nq = (size_t)B * Hq * d;
+    if ((t + 1) % g != 0) {
+        for (size_t e = 0; e < nq; ++e) q_sum[e] += q[e];
+        c->len = t + 1;
+        return CCA_ORACLE_OK;
+    }
+    const long j = t / g, first = t - g + 1;
+    const int d_content = d - d_rope;
+    const double inv_sqrt_d = 1.0 / sqrt((double)d);
+    double *qbar = (double *)malloc(sizeof(double) * (size_t)d);
+    double *p = (double *)malloc(sizeof(double) * (size_t)g);
+    double *wgt = (double *)malloc(sizeof(double) * (size_t)g);
+    for (int b = 0; b < B; ++b)
+        for (int h = 0; h < Hkv; ++h) {
+            const size_t kv = (size_t)b * Hkv + h;
+            for (int i = 0; i < g; ++i) wgt[i] = 0.0;
+            for (int k2 = 0; k2 < r; ++k2) {
+                const size_t qh = ((size_t)b * Hq + h * r + k2) * d;
+                for (int e = 0; e < d; ++e) qbar[e] = (q_sum[qh + e] + q[qh + e]) / g;
+                for (int i = 0; i < g; ++i) {
+                    const long pos = first + i;
+                    p[i] = dot(qbar, c->k_tail + (kv * c->tail_cap + pos % c->tail_cap) * d, d) *
+                           inv_sqrt_d;
+                }
+                softmax_inplace(p, g);
+                for (int i = 0; i < g; ++i) wgt[i] += p[i] / (double)r;
+            }
+            int best = 0;
+            for (int i = 1; i < g; ++i)
+                if (wgt[i] > wgt[best]) best = i;
+            const size_t best_row = kv * c->tail_cap + (first + best) % c->tail_cap;
+            double *kc = c->k_core + (kv * c->core_cap + j) * d;
+            double *vc = c->v_core + (kv * c->core_cap + j) * d;
+            for (int e = 0; e < d; ++e) {
+                double kacc = 0.0, vacc = 0.0;
+                for (int i = 0; i < g; ++i) {
+                    const size_t row = kv * c->tail_cap + (first + i) % c->tail_cap;
+                    kacc += wgt[i] * c->k_tail[row * d + e];
+                    vacc += wgt[i] * c->v_tail[row * d + e];
+                }
+                kc[e] = e < d_content ? kacc : c->k_tail[best_row * d + e];
+                vc[e] = vacc;
+            }
+        }
+    free(qbar);
+    free(p);
+    free(wgt);
+    for (size_t e = 0; e < nq; ++e) q_sum[e] = 0.0;
+    c->len = t + 1;
+    return CCA_ORACLE_OK;
+}
+
 int cca_oracle_decode(const cca_oracle_cache *c, const double *q, double *o)
 {
     if (!cache_ok(c) || c->len <= 0) return CCA_ORACLE_EINVAL;

@@ -76,6 +76,14 @@ typedef struct {
 int cca_oracle_cache_append(cca_oracle_cache *c, const double *q,
                             const double *k, const double *v);
 
+/* LCA variant: append token t = len (ring slot t % tail_cap); q_sum
+ * [B, Hq, d] holds the open group's query sums, to which q is added, or, if
+ * t completes group j = t / g, the group is condensed as cca_oracle_lca_pool
+ * does, with average queries (q_sum + q) / g, into core slot j and q_sum is
+ * zeroed.  Then len = t + 1. */
+int cca_oracle_lca_cache_append(cca_oracle_cache *c, double *q_sum, const double *q,
+                                const double *k, const double *v, int d_rope);
+
 /* Attention of the newest token t = len - 1 with queries q [B, Hq, d] over
  * the cache; writes o [B, Hq, d]. */
 int cca_oracle_decode(const cca_oracle_cache *c, const double *q, double *o);

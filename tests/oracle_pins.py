@@ -388,6 +388,32 @@ def pin_lca_trailing_partial_group(orc):
     np.testing.assert_array_equal(Vc, Vc2)
 
 
+def pin_lca_cache_condenses_as_lca_pool(orc):
+    """The LCA decode cache (推理流程: groups condensed as tokens arrive,
+    with the running sums of the open group's queries) ends with the same
+    core tokens as condensing the whole sequence at once, keeps the open
+    group's query sums, and its decode of token t is row t of the fused
+    attention over those core tokens.  The ring (w + g slots) wraps."""
+    r = _rng(26)
+    B, Hq, Hkv, T, d, g, w, d_rope = 2, 4, 2, 75, 8, 4, 10, 4
+    Q = r.standard_normal((B, Hq, T, d))
+    K = r.standard_normal((B, Hkv, T, d))
+    V = r.standard_normal((B, Hkv, T, d))
+    Kc, Vc = orc.lca_pool(Q, K, V, g, d_rope)
+    m = T // g
+    c = orc.cache(B, Hq, Hkv, d, g, w, core_cap=m + 1)
+    q_sum = np.zeros((B, Hq, d))
+    for t in range(T):
+        c.lca_append(q_sum, Q[:, :, t], K[:, :, t], V[:, :, t], d_rope)
+        if t >= 40:
+            np.testing.assert_allclose(c.decode(Q[:, :, t]),
+                                       orc.attend_rows(Q, K, V, Kc, Vc, g, w, [t])[:, :, 0],
+                                       atol=1e-12)
+    np.testing.assert_allclose(c.k_core[:, :, :m], Kc, atol=1e-12)
+    np.testing.assert_allclose(c.v_core[:, :, :m], Vc, atol=1e-12)
+    np.testing.assert_allclose(q_sum, Q[:, :, m * g:].sum(axis=2), atol=1e-12)
+
+
 # ---------------------------------------------------------------------------
 # fused attention (sections 局部保留模块, 全局-局部模块可微融合)
 # ---------------------------------------------------------------------------

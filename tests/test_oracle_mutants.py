@@ -53,6 +53,13 @@ MUTANTS = [
      "vacc += wgt[i] * Kg[(size_t)i * d + c];", 0),
     ("lca query rows of head 0 only", "Q + (((size_t)b * Hq + h * r + k) * T + first) * d;",
      "Q + (((size_t)b * Hq + h * r) * T + first) * d;", 0),
+    ("lca cache forgets the token's own query", "qbar[e] = (q_sum[qh + e] + q[qh + e]) / g;",
+     "qbar[e] = q_sum[qh + e] / g;", 0),
+    ("lca cache keeps stale sums", "for (size_t e = 0; e < nq; ++e) q_sum[e] = 0.0;",
+     "for (size_t e = 0; e < nq; ++e) q_sum[e] = q_sum[e];", 0),
+    ("lca cache anchor ignores the ring position",
+     "const size_t best_row = kv * c->tail_cap + (first + best) % c->tail_cap;",
+     "const size_t best_row = kv * c->tail_cap + best % c->tail_cap;", 0),
     ("capacity check off by one", "if (t / g >= c->core_cap) return CCA_ORACLE_ECAPACITY;",
      "if (t / g > c->core_cap) return CCA_ORACLE_ECAPACITY;", 0),
 ]
